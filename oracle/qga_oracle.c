@@ -1,0 +1,374 @@
+/*
+ * qga_oracle.c -- the CPU oracle for quantized gradient aggregation.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the slow, obviously-correct
+ * statement of what the GPU library computes.  Only the test suite, the
+ * smoke check of the package entry point and the CPU-baseline leg of the
+ * benchmark may load it.  The CUDA library never links, includes or calls it,
+ * and it shares no header, helper, table or constant with the CUDA sources.
+ *
+ * Build: gcc -std=c11 -O2 -ffp-contract=off -fno-fast-math -fPIC -shared.
+ * On x86-64 every `float` expression below is one IEEE-754 binary32 operation
+ * rounded to nearest-even (SSE arithmetic, FLT_EVAL_METHOD == 0); with
+ * contraction off, no fused multiply-add is ever formed.
+ *
+ * Sources, cited by page title and section:
+ *   [MX]  MXNet pull request #8342 "[WIP] 2bit gradient compression":
+ *         sections "Approach", "Two bit quantization", "Format of compressed
+ *         gradient", "Operators", "Local kvstore".
+ *   [GC]  gradient-compression README (vineeths96), "About The Project" and
+ *         "Results": names QSGDMaxNorm quantization and calls it all-reduce
+ *         compatible; it prints no formula.  The QSGD-MaxNorm steps below are
+ *         this library's definition of the method (global max-norm scale,
+ *         s = 2^(b-1)-1 levels, stochastic rounding, signed b-bit codes).
+ *   [SC11] J. Salmon, M. Moraes, R. Dror, D. Shaw, "Parallel Random Numbers:
+ *         As Easy as 1, 2, 3", SC'11 -- the Philox4x32-10 generator.
+ *
+ * Pinning (what checks this file against something other than itself) is
+ * done by the CPU tests: the worked example printed in [MX] "Format of
+ * compressed gradient", exhaustive round trips, IEEE rounding bounds checked
+ * in exact rational arithmetic, error-feedback telescoping, closed-form
+ * aggregates, published Philox known-answer vectors and statistical
+ * properties of the stochastic rounding.  Every function here has at least
+ * one such pin; none is "parity unpinned".
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------ */
+/* bit views of binary32                                               */
+/* ------------------------------------------------------------------ */
+static uint32_t bits_of(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return u;
+}
+
+static float float_of(uint32_t u)
+{
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* ------------------------------------------------------------------ */
+/* 2-bit threshold quantization with error feedback  [MX]              */
+/* ------------------------------------------------------------------ */
+
+/* [MX] "Format of compressed gradient": two thresholds, the original size,
+ * then one 32-bit word per (up to) 16 original elements. */
+int64_t oracle_2bit_words(int64_t n)
+{
+    return 3 + (n + 15) / 16;
+}
+
+/* [MX] "Two bit quantization": a value at or above the positive threshold
+ * gets code 01, a value at or below the negative threshold gets code 10,
+ * anything else gets code 00.  The positive test is taken first. */
+static uint32_t two_bit_code(float value, float neg_thr, float pos_thr)
+{
+    if (value >= pos_thr)
+        return 1u;
+    if (value <= neg_thr)
+        return 2u;
+    return 0u;
+}
+
+/* Value a code stands for: the threshold that produced it, or zero.  The
+ * header keeps the thresholds because they "are required to dequantize"
+ * ([MX] "Format of compressed gradient").  Code 11 is never produced; it
+ * decodes to zero. */
+static float two_bit_value(uint32_t code, float neg_thr, float pos_thr)
+{
+    if (code == 1u)
+        return pos_thr;
+    if (code == 2u)
+        return neg_thr;
+    return 0.0f;
+}
+
+/* Shift that puts the code of the element at position p (0..15) of its word
+ * into place: the first element of a word sits in the two most significant
+ * bits (the worked example's bit string 00 01 00 10 01 00 00 10 0...0). */
+static int two_bit_shift(int64_t e)
+{
+    return 30 - 2 * (int)(e % 16);
+}
+
+static void write_2bit_header(uint32_t *compr, int64_t n, float neg_thr, float pos_thr)
+{
+    compr[0] = bits_of(neg_thr);
+    compr[1] = bits_of(pos_thr);
+    compr[2] = bits_of((float)n); /* the example prints n as the float 8 */
+}
+
+/* One element of the error-feedback step ([MX] "Approach", "Two bit
+ * quantization"): the stored residual is added to the gradient, the sum is
+ * coded, and what the code does not carry stays in the residual. */
+static uint32_t quantize_one(float grad, float *residual, float neg_thr, float pos_thr)
+{
+    float with_residual = grad + *residual;
+    uint32_t code = two_bit_code(with_residual, neg_thr, pos_thr);
+    *residual = with_residual - two_bit_value(code, neg_thr, pos_thr);
+    return code;
+}
+
+/* quantize_2bit(grad, residual, compr, neg_threshold, pos_threshold) of
+ * [MX] "Operators", fp32 gradient.  compr holds oracle_2bit_words(n) words. */
+void oracle_quantize_2bit(const float *grad, float *residual, uint32_t *compr,
+                          int64_t n, float neg_thr, float pos_thr)
+{
+    write_2bit_header(compr, n, neg_thr, pos_thr);
+    for (int64_t w = 0; w < (n + 15) / 16; ++w)
+        compr[3 + w] = 0u;
+    for (int64_t e = 0; e < n; ++e) {
+        uint32_t code = quantize_one(grad[e], &residual[e], neg_thr, pos_thr);
+        compr[3 + e / 16] |= code << two_bit_shift(e);
+    }
+}
+
+/* bfloat16 is the upper half of a binary32 bit pattern, so widening it is
+ * exact: append sixteen zero bits. */
+static float widen_bf16(uint16_t h)
+{
+    return float_of((uint32_t)h << 16);
+}
+
+/* The same operator for a bfloat16 gradient and an fp32 residual. */
+void oracle_quantize_2bit_bf16(const uint16_t *grad, float *residual, uint32_t *compr,
+                               int64_t n, float neg_thr, float pos_thr)
+{
+    write_2bit_header(compr, n, neg_thr, pos_thr);
+    for (int64_t w = 0; w < (n + 15) / 16; ++w)
+        compr[3 + w] = 0u;
+    for (int64_t e = 0; e < n; ++e) {
+        uint32_t code = quantize_one(widen_bf16(grad[e]), &residual[e], neg_thr, pos_thr);
+        compr[3 + e / 16] |= code << two_bit_shift(e);
+    }
+}
+
+static uint32_t two_bit_code_at(const uint32_t *compr, int64_t e)
+{
+    return (compr[3 + e / 16] >> two_bit_shift(e)) & 3u;
+}
+
+/* dequantize_2bit(compr, decompr) of [MX] "Operators": every element becomes
+ * the value of its code, with the thresholds read from the record's header.
+ * n is the caller's element count (the header's float copy of n is not exact
+ * above 2^24). */
+void oracle_dequantize_2bit(const uint32_t *compr, float *out, int64_t n)
+{
+    float neg_thr = float_of(compr[0]);
+    float pos_thr = float_of(compr[1]);
+    for (int64_t e = 0; e < n; ++e)
+        out[e] = two_bit_value(two_bit_code_at(compr, e), neg_thr, pos_thr);
+}
+
+/* The receiver's merge of [MX] "Local kvstore": every worker's record is
+ * dequantized with its own header and the results are summed.  The sum
+ * starts from +0 and adds the workers in the order 0, 1, ..., W-1. */
+void oracle_dequant_accumulate_2bit(const uint32_t *const *compr, int W, float *out, int64_t n)
+{
+    for (int64_t e = 0; e < n; ++e) {
+        float sum = 0.0f;
+        for (int w = 0; w < W; ++w) {
+            float neg_thr = float_of(compr[w][0]);
+            float pos_thr = float_of(compr[w][1]);
+            sum = sum + two_bit_value(two_bit_code_at(compr[w], e), neg_thr, pos_thr);
+        }
+        out[e] = sum;
+    }
+}
+
+/* Bucket of T tensors: the compressed bucket is the T standalone records one
+ * after the other, each padded to whole words as every record is. */
+int64_t oracle_2bit_bucket_words(const int64_t *n, int T)
+{
+    int64_t words = 0;
+    for (int t = 0; t < T; ++t)
+        words += oracle_2bit_words(n[t]);
+    return words;
+}
+
+/* grads[t] points at an fp32 array when grad_is_bf16 == 0, else at bf16. */
+void oracle_quantize_2bit_bucket(const void *const *grads, float *const *residuals,
+                                 const int64_t *n, const float *neg_thr, const float *pos_thr,
+                                 int T, int grad_is_bf16, uint32_t *compr)
+{
+    int64_t offset = 0;
+    for (int t = 0; t < T; ++t) {
+        if (grad_is_bf16)
+            oracle_quantize_2bit_bf16((const uint16_t *)grads[t], residuals[t], compr + offset,
+                                      n[t], neg_thr[t], pos_thr[t]);
+        else
+            oracle_quantize_2bit((const float *)grads[t], residuals[t], compr + offset,
+                                 n[t], neg_thr[t], pos_thr[t]);
+        offset += oracle_2bit_words(n[t]);
+    }
+}
+
+/* Merge of W compressed buckets into one fp32 buffer holding the T tensors
+ * one after the other. */
+void oracle_dequant_accumulate_2bit_bucket(const uint32_t *const *compr, int W,
+                                           const int64_t *n, int T, float *out)
+{
+    const uint32_t *records[64];
+    int64_t word_offset = 0, elem_offset = 0;
+    for (int t = 0; t < T; ++t) {
+        for (int w = 0; w < W; ++w)
+            records[w] = compr[w] + word_offset;
+        oracle_dequant_accumulate_2bit(records, W, out + elem_offset, n[t]);
+        word_offset += oracle_2bit_words(n[t]);
+        elem_offset += n[t];
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* Philox4x32-10  [SC11]                                               */
+/* ------------------------------------------------------------------ */
+
+/* One round: two 32x32->64 products of the even counter words with the
+ * round multipliers; the high halves are mixed with the odd words and the
+ * key, the low halves move into the odd slots. */
+static void philox_round(uint32_t ctr[4], const uint32_t key[2])
+{
+    uint64_t p0 = (uint64_t)0xD2511F53u * ctr[0];
+    uint64_t p1 = (uint64_t)0xCD9E8D57u * ctr[2];
+    uint32_t next[4];
+    next[0] = (uint32_t)(p1 >> 32) ^ ctr[1] ^ key[0];
+    next[1] = (uint32_t)p1;
+    next[2] = (uint32_t)(p0 >> 32) ^ ctr[3] ^ key[1];
+    next[3] = (uint32_t)p0;
+    memcpy(ctr, next, sizeof next);
+}
+
+/* Ten rounds; the key is advanced by the Weyl increments (golden ratio and
+ * sqrt(3)-1 in 0.32 fixed point) before every round after the first. */
+void oracle_philox4x32_10(const uint32_t counter[4], const uint32_t key_in[2], uint32_t out[4])
+{
+    uint32_t ctr[4] = {counter[0], counter[1], counter[2], counter[3]};
+    uint32_t key[2] = {key_in[0], key_in[1]};
+    for (int round = 0; round < 10; ++round) {
+        if (round > 0) {
+            key[0] += 0x9E3779B9u;
+            key[1] += 0xBB67AE85u;
+        }
+        philox_round(ctr, key);
+    }
+    memcpy(out, ctr, sizeof ctr);
+}
+
+/* ------------------------------------------------------------------ */
+/* QSGD-MaxNorm, b bits  ([GC] names it; steps as defined above)       */
+/* ------------------------------------------------------------------ */
+
+/* The global scale M: the largest |g| over every worker's buffer.  A NaN
+ * element never compares greater, so it is skipped. */
+float oracle_qsgd_mn_max(const float *const *grad, int W, int64_t n)
+{
+    float m = 0.0f;
+    for (int w = 0; w < W; ++w)
+        for (int64_t e = 0; e < n; ++e) {
+            float a = fabsf(grad[w][e]);
+            if (a > m)
+                m = a;
+        }
+    return m;
+}
+
+/* The uniform draw of element e: Philox4x32-10 keyed by the 64-bit seed
+ * (low word first), counter (e/4 low word, e/4 high word, 0, 0); element e
+ * takes output word e mod 4, keeps its top 24 bits and scales by 2^-24, so
+ * u is a multiple of 2^-24 in [0, 1 - 2^-24], exact in binary32. */
+float oracle_qsgd_uniform(uint64_t seed, int64_t e)
+{
+    uint64_t block = (uint64_t)e / 4;
+    uint32_t ctr[4] = {(uint32_t)block, (uint32_t)(block >> 32), 0u, 0u};
+    uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+    uint32_t out[4];
+    oracle_philox4x32_10(ctr, key, out);
+    return (float)(out[e % 4] >> 8) * 0x1p-24f;
+}
+
+static int qsgd_levels(int b)
+{
+    return (1 << (b - 1)) - 1;
+}
+
+/* The signed level of one element: scale |g| by the global max, stretch to
+ * s levels, add the uniform draw and round down, cap at s, restore the sign.
+ * Each arithmetic step is one binary32 operation in this order:
+ *   t = ((|g| / M) * s) + u,   q = sign(g) * min(floor(t), s).
+ * A non-finite t (M == 0, or non-finite input) gives level 0. */
+int32_t oracle_qsgd_level(float grad, float M, int b, uint64_t seed, int64_t e)
+{
+    int s = qsgd_levels(b);
+    float u = oracle_qsgd_uniform(seed, e);
+    float scaled = fabsf(grad) / M;
+    float stretched = scaled * (float)s;
+    float t = stretched + u;
+    if (!isfinite(t))
+        return 0;
+    float level = floorf(t);
+    if (level > (float)s)
+        level = (float)s;
+    int32_t q = (int32_t)level;
+    return grad < 0.0f ? -q : q;
+}
+
+int64_t oracle_qsgd_words(int64_t n, int b)
+{
+    return 3 + (n * b + 31) / 32;
+}
+
+/* Record: header [M, b, n] as binary32, then 32/b two's-complement codes of
+ * b bits per word, the first element of a word in its most significant bits
+ * (the same order as the 2-bit format), unused tail codes zero. */
+void oracle_qsgd_mn_quantize(const float *grad, uint32_t *compr, int64_t n, int b,
+                             uint64_t seed, float M)
+{
+    int per_word = 32 / b;
+    uint32_t mask = (1u << b) - 1u;
+    compr[0] = bits_of(M);
+    compr[1] = bits_of((float)b);
+    compr[2] = bits_of((float)n);
+    for (int64_t w = 0; w < (n * b + 31) / 32; ++w)
+        compr[3 + w] = 0u;
+    for (int64_t e = 0; e < n; ++e) {
+        int32_t q = oracle_qsgd_level(grad[e], M, b, seed, e);
+        uint32_t code = (uint32_t)q & mask;
+        int shift = 32 - b * (int)(e % per_word + 1);
+        compr[3 + e / per_word] |= code << shift;
+    }
+}
+
+/* Level of element e read back from a record: the b-bit field, sign-extended. */
+static int32_t qsgd_level_at(const uint32_t *compr, int64_t e, int b)
+{
+    int per_word = 32 / b;
+    int shift = 32 - b * (int)(e % per_word + 1);
+    uint32_t code = (compr[3 + e / per_word] >> shift) & ((1u << b) - 1u);
+    int32_t q = (int32_t)code;
+    if (code >= (1u << (b - 1)))
+        q -= (int32_t)(1u << b);
+    return q;
+}
+
+/* Aggregate of W records: the integer levels are summed (exact), then scaled
+ * once by M / s, with M read from worker 0's header (every worker quantized
+ * with the same global M).  This is the sum-then-scale form that makes the
+ * scheme all-reduce compatible ([GC] "About The Project"). */
+void oracle_qsgd_mn_dequant_accumulate(const uint32_t *const *compr, int W, float *out,
+                                       int64_t n, int b)
+{
+    float M = float_of(compr[0][0]);
+    float step = M / (float)qsgd_levels(b);
+    for (int64_t e = 0; e < n; ++e) {
+        int32_t sum = 0;
+        for (int w = 0; w < W; ++w)
+            sum += qsgd_level_at(compr[w], e, b);
+        out[e] = (float)sum * step;
+    }
+}
