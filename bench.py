@@ -1,0 +1,422 @@
+#!/usr/bin/env python3
+"""Benchmark of the quantized-gradient-aggregation hot path on B200.
+
+One step = one pass of the error-feedback 2-bit path of the VGG16-sized
+workload: each of W = 8 simulated workers quantizes its own n = 138,357,544
+element fp32 gradient against its own residual (fused add / code / residual
+update / pack, ``qga_quantize_2bit``), then the 8 packed streams are merged
+into one fp32 aggregate (``qga_dequant_accumulate_2bit``).  Gradients are
+seeded Laplace(0, 1e-3) draws, 5 iterations' worth resident in HBM and
+cycled, residuals carried from step to step; thresholds +-2e-3.
+
+``value`` is gradient elements aggregated per second over the whole job
+(W * n per step per GPU), timed with CUDA events on the launching stream,
+max over ranks.  Every buffer is larger than L2, so no flush is needed.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl qga|reference]
+
+``--impl reference`` times the CPU oracle (single-threaded C) as it stands on
+a bounded sample of the same workload.  Under torchrun with N > 1 each rank
+runs its own replica (weak scaling, no collective on the data path).
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import datetime
+import glob
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "2-bit quantize+residual+pack Gelem/s and HBM GB/s (% of peak), n=138M fp32"
+WORKLOAD = "vgg16-8w"
+QUANT_BYTES_PER_ELEM = 12.25        # read g 4 + read r 4 + write r 4 + write codes 0.25
+FALLBACK_HBM_GBS = 6650.0
+
+# dram__bytes_read.sum + dram__bytes_write.sum per element of the quantize
+# kernel, from the ncu capture in profiles/, keyed by the hash of the CUDA
+# sources it was taken on (reported as null once the kernel has changed).
+MEASURED_TRAFFIC = {}
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=300)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["qga", "reference"], default="qga")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    # smaller cases of the same step, for profiler captures (not bench lines)
+    p.add_argument("--n", type=int, default=None, help="elements per worker (default: workload n)")
+    p.add_argument("--iterations", type=int, default=None, help="resident gradient sets")
+    return p.parse_args()
+
+
+def csrc_hash():
+    h = hashlib.sha256()
+    pkg = os.path.join(ROOT, "quantized_gradient_aggregation_b200", "csrc")
+    for path in sorted(glob.glob(os.path.join(pkg, "*.cu*"))):
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def workload_config(w, n_gpus):
+    return {
+        "workload": (f"{w.name}: W={w.workers} simulated workers x n={w.n:,} fp32, "
+                     f"g~Laplace(0,{w.scale:g}) (seeded synthetic, {w.iterations} iterations "
+                     f"resident and cycled), residual carried, thresholds {w.neg_thr:g}/{w.pos_thr:g}; "
+                     "step = 8 quantize + 1 merge of 8 packed streams"),
+        "n": w.n,
+        "workers": w.workers,
+        "l2": "every buffer (553 MB per gradient) is larger than the 126 MB L2; no flush",
+        "parallelism": f"replicas x{n_gpus} (weak scaling, no data-path collective)",
+    }
+
+
+# ------------------------------------------------------------ clocks ----
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def __init__(self, gpu_id):
+        self.out = tempfile.TemporaryFile(mode="w+")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={gpu_id}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.seek(0)
+        sm, smax, reasons, n = [], [], set(), 0
+        for line in self.out:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            n += 1
+            for name, flag in zip(self.REASONS, parts[5:9]):
+                if flag.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": n}
+
+
+def gpu_id_for(dev_index):
+    import torch
+    props = torch.cuda.get_device_properties(dev_index)
+    uuid = getattr(props, "uuid", None)
+    if uuid is not None:
+        s = str(uuid)
+        return s if s.startswith("GPU-") else "GPU-" + s
+    return str(dev_index)
+
+
+# ------------------------------------------------------------ oracle ----
+
+def oracle_step_sample(n_s, seed=0):
+    """Host inputs for a bounded sample of the workload (first n_s elements
+    of each worker's gradient)."""
+    import numpy as np
+    import workloads
+    w = workloads.WORKLOADS[WORKLOAD]
+    grads = [workloads.gradient(w, k, 0, device="cpu", n=n_s).numpy() for k in range(w.workers)]
+    res = [np.zeros(n_s, np.float32) for _ in range(w.workers)]
+    return w, grads, res
+
+
+def time_oracle(n_s, min_seconds, max_steps=None, warmup=0):
+    """Oracle steps (W quantizes + 1 merge) on n_s elements per worker."""
+    import oracle
+    L = oracle.lib()
+    w, grads, res = oracle_step_sample(n_s)
+    ptrs = (ctypes.c_void_p * w.workers)()
+
+    def step():
+        recs = []
+        for k in range(w.workers):
+            c, res[k] = oracle.quantize_2bit(grads[k], res[k], w.neg_thr, w.pos_thr, L)
+            recs.append(c)
+        oracle.dequant_accumulate_2bit(recs, n_s, L)
+
+    for _ in range(warmup):
+        step()
+    t0 = time.perf_counter()
+    steps = 0
+    while True:
+        step()
+        steps += 1
+        el = time.perf_counter() - t0
+        if (max_steps is not None and steps >= max_steps) or (max_steps is None and el >= min_seconds):
+            break
+    el = time.perf_counter() - t0
+    del ptrs
+    return steps, el, w
+
+
+def cpu_baseline(n_s=1 << 24, min_seconds=10.0):
+    steps, el, w = time_oracle(n_s, min_seconds)
+    elems = steps * w.workers * n_s
+    return {"value": elems / el / 1e9, "unit": "Gelem/s", "cores": 1, "kind": "oracle",
+            "sample": (f"{steps} oracle steps of {w.workers} workers x {n_s:,} elements "
+                       f"(first {n_s:,} of each worker's gradient) quantize + merge, "
+                       f"{el:.1f} s single-threaded; host has {len(os.sched_getaffinity(0))} cores")}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    # per-step sample sized so the whole run stays near a minute (the oracle
+    # takes about 15 ns per element per worker, merge included)
+    budget_s = 60.0 / max(1, args.steps + args.warmup)
+    n_s = int(min(1 << 22, max(1 << 14, budget_s / (8 * 15e-9)))) & ~15
+    steps, el, w = time_oracle(n_s, 0.0, max_steps=args.steps, warmup=args.warmup)
+    value = steps * w.workers * n_s / el / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "Gelem/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded Laplace draws)", "config": workload_config(w, args.gpus),
+        "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": "Gelem/s", "cores": 1, "kind": "oracle",
+                         "sample": (f"each step: {w.workers} workers x first {n_s:,} elements of "
+                                    "the workload, quantize + merge, single-threaded C oracle; host "
+                                    f"has {len(os.sched_getaffinity(0))} cores")},
+        "e2e": {"value": value, "unit": "Gelem/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------- GPU ----
+
+def run_qga(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import quantized_gradient_aggregation_b200 as q
+    import workloads
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = workloads.WORKLOADS[WORKLOAD]
+    if args.n is not None or args.iterations is not None:
+        import dataclasses
+        w = dataclasses.replace(w, n=args.n or w.n, iterations=args.iterations or w.iterations,
+                                name=w.name + "-small")
+    n, W, iters = w.n, w.workers, w.iterations
+    L = q.lib()
+
+    grads = [[workloads.gradient(w, k, it, device=dev) for k in range(W)] for it in range(iters)]
+    res = [torch.zeros(n, device=dev) for _ in range(W)]
+    words = q.qga_2bit_words(n)
+    comprs = [torch.empty(words, dtype=torch.int32, device=dev) for _ in range(W)]
+    out = torch.empty(n, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    cptrs = (ctypes.c_void_p * W)(*[c.data_ptr() for c in comprs])
+    cpp = ctypes.cast(cptrs, ctypes.POINTER(ctypes.c_void_p))
+    neg, pos = w.neg_thr, w.pos_thr
+
+    def quant(it, k):
+        st = L.qga_quantize_2bit(ctypes.c_void_p(grads[it][k].data_ptr()),
+                                 ctypes.c_void_p(res[k].data_ptr()),
+                                 ctypes.c_void_p(comprs[k].data_ptr()), n, neg, pos, sp)
+        if st:
+            raise q.QGAError(st, "qga_quantize_2bit")
+
+    def merge():
+        st = L.qga_dequant_accumulate_2bit(cpp, W, ctypes.c_void_p(out.data_ptr()), n, sp)
+        if st:
+            raise q.QGAError(st, "qga_dequant_accumulate_2bit")
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    sampler = ClockSampler(gpu_id_for(local_rank))
+    time.sleep(0.3)
+    for s in range(args.warmup):
+        for k in range(W):
+            quant(s % iters, k)
+        merge()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+
+    K = args.steps
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    q_ev = [(ev(), ev()) for _ in range(K * W)]
+    m_ev = [(ev(), ev()) for _ in range(K)]
+    start, end = ev(), ev()
+    start.record(stream)
+    for s in range(K):
+        it = (args.warmup + s) % iters
+        for k in range(W):
+            a, b = q_ev[s * W + k]
+            a.record(stream)
+            quant(it, k)
+            b.record(stream)
+        a, b = m_ev[s]
+        a.record(stream)
+        merge()
+        b.record(stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+
+    total_ms = start.elapsed_time(end)
+    quant_ms = statistics.fmean(a.elapsed_time(b) for a, b in q_ev)
+    merge_ms = statistics.fmean(a.elapsed_time(b) for a, b in m_ev)
+    t = torch.tensor([total_ms, quant_ms, merge_ms], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, quant_ms, merge_ms = t.tolist()
+
+    e2e = None if args.no_e2e else run_e2e(args, w, grads[0], res, comprs, out, quant, merge,
+                                           stream, world, dev)
+    del grads
+
+    if rank != 0:
+        return
+    peak, peak_kind = measured_peaks()
+    quant_gbs = QUANT_BYTES_PER_ELEM * n / (quant_ms * 1e-3) / 1e9
+    merge_gbs = (0.25 * W + 4) * n / (merge_ms * 1e-3) / 1e9
+    traffic_per_elem = MEASURED_TRAFFIC.get(csrc_hash())
+    line = {
+        "metric": METRIC,
+        "value": world * W * n * K / (total_ms * 1e-3) / 1e9,
+        "unit": "Gelem/s",
+        "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": total_ms / K,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded Laplace(0,1e-3) gradients generated on the GPU)",
+        "config": workload_config(w, world),
+        "roofline": {"bound": "hbm", "kernel": "qga_quantize_2bit (quantize_2bit_kernel<float>)",
+                     "achieved": quant_gbs, "peak": peak, "unit": "GB/s", "frac": quant_gbs / peak,
+                     "peak_source": f"{peak_kind} HBM copy rate",
+                     "bytes_per_elem": QUANT_BYTES_PER_ELEM, "elems_per_launch": n,
+                     "avg_launch_us": quant_ms * 1e3,
+                     "traffic": None if traffic_per_elem is None else traffic_per_elem * n},
+        "kernels": {
+            "quantize_2bit": {"us": quant_ms * 1e3, "gelem_s": n / (quant_ms * 1e-3) / 1e9,
+                              "gb_s": quant_gbs, "frac_of_peak": quant_gbs / peak,
+                              "frac_of_8TBs": quant_gbs / 8000.0},
+            "dequant_accumulate_2bit_w8": {"us": merge_ms * 1e3,
+                                           "gelem_s": n / (merge_ms * 1e-3) / 1e9,
+                                           "gb_s": merge_gbs, "frac_of_peak": merge_gbs / peak,
+                                           "frac_of_8TBs": merge_gbs / 8000.0},
+        },
+        "gpu_launches": K * (W + 1),
+        "clocks": clocks,
+        "csrc": csrc_hash(),
+    }
+    if e2e is not None:
+        line["e2e"] = e2e
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
+    print(json.dumps(line), flush=True)
+
+
+def run_e2e(args, w, dev_grads, res, comprs, out, quant, merge, stream, world, dev):
+    """Same step with the gradients arriving from pinned host memory and the
+    aggregate read back, copies inside the timed region."""
+    import torch
+    import torch.distributed as dist
+    n, W = w.n, w.workers
+    host = [torch.empty(n, dtype=torch.float32, pin_memory=True) for _ in range(W)]
+    for k in range(W):
+        host[k].copy_(dev_grads[k], non_blocking=False)
+    host_out = torch.empty(n, dtype=torch.float32, pin_memory=True)
+    K = max(3, min(args.steps, 10))
+
+    def step():
+        for k in range(W):
+            dev_grads[k].copy_(host[k], non_blocking=True)
+            quant(0, k)
+        merge()
+        host_out.copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(K):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b)
+    t = torch.tensor([ms], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = t.item()
+    return {"value": world * W * n * K / (ms * 1e-3) / 1e9, "unit": "Gelem/s",
+            "h2d_bytes_per_step": W * n * 4, "d2h_bytes_per_step": n * 4, "steps": K,
+            "path": "pinned host gradients -> cudaMemcpyAsync -> qga_quantize_2bit x8 -> "
+                    "qga_dequant_accumulate_2bit -> pinned host aggregate"}
+
+
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_qga(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

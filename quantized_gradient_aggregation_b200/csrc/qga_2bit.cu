@@ -1,0 +1,181 @@
+// qga_2bit.cu -- single-tensor 2-bit threshold kernels and their C ABI:
+// quantize (fp32 / bf16 gradient), dequantize, and the W-worker merge.
+//
+// MXNet pull request #8342 "[WIP] 2bit gradient compression": "Operators"
+// (create_2bit / quantize_2bit / dequantize_2bit), "Format of compressed
+// gradient" (header [neg, pos, n] then 16 codes per word) and "Local kvstore"
+// (the receiver dequantizes every worker's gradient and sums them).
+//
+// Each kernel is one pass over HBM with a persistent grid (every SM filled
+// once; warps stride over 512-element tiles).  Nothing is filled or cleared
+// by a separate launch: the quantize kernel writes every payload word
+// (including the zero tail codes) and its block 0 writes the header.
+
+#include "qga_2bit_tiles.cuh"
+
+namespace qga {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarpsPerBlock = kThreads / kWarp;
+
+__device__ __forceinline__ int64_t first_tile() { return (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5); }
+__device__ __forceinline__ int64_t tile_stride() { return (int64_t)gridDim.x * kWarpsPerBlock; }
+
+template <typename G, bool kVec>
+__global__ void __launch_bounds__(kThreads)
+    quantize_2bit_kernel(const G *__restrict__ grad, float *__restrict__ residual,
+                         uint32_t *__restrict__ compr, int64_t n, float neg, float pos)
+{
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        compr[0] = bits_from_f32(neg);
+        compr[1] = bits_from_f32(pos);
+        compr[2] = bits_from_f32(__ll2float_rn(n));
+    }
+    const int lane = threadIdx.x & (kWarp - 1);
+    const int64_t tiles = (n + kTileElems - 1) / kTileElems;
+    for (int64_t t = first_tile(); t < tiles; t += tile_stride())
+        quantize_2bit_tile<G, kVec>(grad, residual, compr + 3, n, t, neg, pos, lane);
+}
+
+template <bool kVec>
+__global__ void __launch_bounds__(kThreads)
+    dequantize_2bit_kernel(const uint32_t *__restrict__ compr, float *__restrict__ out, int64_t n)
+{
+    const float neg = f32_from_bits(compr[0]);
+    const float pos = f32_from_bits(compr[1]);
+    const int lane = threadIdx.x & (kWarp - 1);
+    const int64_t tiles = (n + kTileElems - 1) / kTileElems;
+    for (int64_t t = first_tile(); t < tiles; t += tile_stride())
+        dequantize_2bit_tile<kVec>(compr + 3, out, n, t, neg, pos, lane);
+}
+
+struct RecordSet {
+    const uint32_t *rec[QGA_MAX_WORKERS];
+};
+
+template <bool kVec>
+__global__ void __launch_bounds__(kThreads)
+    dequant_accumulate_2bit_kernel(const __grid_constant__ RecordSet set, int W,
+                                   float *__restrict__ out, int64_t n)
+{
+    __shared__ const uint32_t *s_payload[QGA_MAX_WORKERS];
+    __shared__ float s_neg[QGA_MAX_WORKERS], s_pos[QGA_MAX_WORKERS];
+    if (threadIdx.x < W) {
+        const uint32_t *r = set.rec[threadIdx.x];
+        s_payload[threadIdx.x] = r + 3;
+        s_neg[threadIdx.x] = f32_from_bits(r[0]);
+        s_pos[threadIdx.x] = f32_from_bits(r[1]);
+    }
+    __syncthreads();
+    const int lane = threadIdx.x & (kWarp - 1);
+    const int64_t tiles = (n + kTileElems - 1) / kTileElems;
+    for (int64_t t = first_tile(); t < tiles; t += tile_stride())
+        dequant_accumulate_2bit_tile<kVec>(
+            W, [&](int w) { return s_payload[w]; }, [&](int w) { return s_neg[w]; },
+            [&](int w) { return s_pos[w]; }, out, n, t, lane);
+}
+
+std::atomic<int> occ_q_f32_v[64], occ_q_f32_s[64], occ_q_bf16_v[64], occ_q_bf16_s[64];
+std::atomic<int> occ_dq_v[64], occ_dq_s[64], occ_acc_v[64], occ_acc_s[64];
+
+unsigned tiles_grid(int64_t n, int resident)
+{
+    const int64_t tiles = (n + kTileElems - 1) / kTileElems;
+    return grid_for((tiles + kWarpsPerBlock - 1) / kWarpsPerBlock, resident);
+}
+
+template <typename G>
+int launch_quantize(const G *grad, float *residual, uint32_t *compr, int64_t n, float neg, float pos,
+                    cudaStream_t stream, std::atomic<int> *occ_v, std::atomic<int> *occ_s)
+{
+    if (n < 0 || compr == nullptr || !aligned(compr, 4) || !finite_f32(neg) || !finite_f32(pos))
+        return QGA_ERR_INVALID_ARG;
+    if (n > 0 && (grad == nullptr || residual == nullptr || !aligned(grad, sizeof(G)) ||
+                  !aligned(residual, 4)))
+        return QGA_ERR_INVALID_ARG;
+    const bool vec = aligned(grad, GradLoad<G>::kVecAlign) && aligned(residual, 16);
+    if (vec) {
+        auto k = quantize_2bit_kernel<G, true>;
+        k<<<tiles_grid(n, resident_blocks(k, kThreads, occ_v)), kThreads, 0, stream>>>(
+            grad, residual, compr, n, neg, pos);
+    } else {
+        auto k = quantize_2bit_kernel<G, false>;
+        k<<<tiles_grid(n, resident_blocks(k, kThreads, occ_s)), kThreads, 0, stream>>>(
+            grad, residual, compr, n, neg, pos);
+    }
+    return launch_status();
+}
+
+} // namespace
+} // namespace qga
+
+using namespace qga;
+
+extern "C" int64_t qga_2bit_words(int64_t n)
+{
+    if (n < 0)
+        return QGA_ERR_INVALID_ARG;
+    return 3 + (n + 15) / 16;
+}
+
+extern "C" int qga_quantize_2bit(const float *grad, float *residual, uint32_t *compr, int64_t n,
+                                 float neg_threshold, float pos_threshold, cudaStream_t stream)
+{
+    return launch_quantize<float>(grad, residual, compr, n, neg_threshold, pos_threshold, stream,
+                                  occ_q_f32_v, occ_q_f32_s);
+}
+
+extern "C" int qga_quantize_2bit_bf16(const uint16_t *grad, float *residual, uint32_t *compr,
+                                      int64_t n, float neg_threshold, float pos_threshold,
+                                      cudaStream_t stream)
+{
+    return launch_quantize<uint16_t>(grad, residual, compr, n, neg_threshold, pos_threshold,
+                                     stream, occ_q_bf16_v, occ_q_bf16_s);
+}
+
+extern "C" int qga_dequantize_2bit(const uint32_t *compr, float *out, int64_t n,
+                                   cudaStream_t stream)
+{
+    if (n < 0 || compr == nullptr || !aligned(compr, 4))
+        return QGA_ERR_INVALID_ARG;
+    if (n == 0)
+        return QGA_OK;
+    if (out == nullptr || !aligned(out, 4))
+        return QGA_ERR_INVALID_ARG;
+    if (aligned(out, 16)) {
+        auto k = dequantize_2bit_kernel<true>;
+        k<<<tiles_grid(n, resident_blocks(k, kThreads, occ_dq_v)), kThreads, 0, stream>>>(compr, out, n);
+    } else {
+        auto k = dequantize_2bit_kernel<false>;
+        k<<<tiles_grid(n, resident_blocks(k, kThreads, occ_dq_s)), kThreads, 0, stream>>>(compr, out, n);
+    }
+    return launch_status();
+}
+
+extern "C" int qga_dequant_accumulate_2bit(const uint32_t *const *compr, int num_workers,
+                                           float *out, int64_t n, cudaStream_t stream)
+{
+    if (n < 0 || compr == nullptr || num_workers < 1 || num_workers > QGA_MAX_WORKERS)
+        return QGA_ERR_INVALID_ARG;
+    RecordSet set{};
+    for (int w = 0; w < num_workers; ++w) {
+        if (compr[w] == nullptr || !aligned(compr[w], 4))
+            return QGA_ERR_INVALID_ARG;
+        set.rec[w] = compr[w];
+    }
+    if (n == 0)
+        return QGA_OK;
+    if (out == nullptr || !aligned(out, 4))
+        return QGA_ERR_INVALID_ARG;
+    if (aligned(out, 16)) {
+        auto k = dequant_accumulate_2bit_kernel<true>;
+        k<<<tiles_grid(n, resident_blocks(k, kThreads, occ_acc_v)), kThreads, 0, stream>>>(
+            set, num_workers, out, n);
+    } else {
+        auto k = dequant_accumulate_2bit_kernel<false>;
+        k<<<tiles_grid(n, resident_blocks(k, kThreads, occ_acc_s)), kThreads, 0, stream>>>(
+            set, num_workers, out, n);
+    }
+    return launch_status();
+}

@@ -1,0 +1,274 @@
+// qga_bucket.cu -- the ragged bucket launcher: T tensors of different sizes,
+// each with its own thresholds, quantized (or merged) in ONE launch.
+//
+// The compressed bucket is the T standalone records of MXNet pull request
+// #8342 "[WIP] 2bit gradient compression" ("Format of compressed gradient")
+// one after the other, so a bucket can be split back into per-tensor records
+// without copying.
+//
+// Work distribution.  Each tensor is cut into chunks of 8192 elements (16
+// warp tiles; a tensor of n = 0 still owns one chunk, which writes its
+// header).  The host numbers the chunks of all tensors consecutively and
+// passes the descriptor table BY VALUE as a kernel parameter (no device
+// table, no allocation, no copy): a persistent grid strides over the chunk
+// numbers, and each block finds its tensor by a binary search over the
+// table's first-chunk column.  Tables over 256 tensors are split into
+// several launches.
+
+#include "qga_2bit_tiles.cuh"
+
+namespace qga {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarpsPerBlock = kThreads / kWarp;
+constexpr int kChunkTiles = 16;
+constexpr int64_t kChunkElems = (int64_t)kChunkTiles * kTileElems;
+constexpr int kMaxRows = 256;
+
+struct QuantRow {
+    const void *grad;
+    float *residual;
+    int64_t n;
+    int64_t word_off;    // record start within the compressed bucket
+    int64_t chunk_begin; // number of this tensor's first chunk within the launch
+    float neg, pos;
+    int vec;             // grad and residual aligned for vector access
+};
+
+struct QuantTable {
+    int T;
+    int64_t total_chunks;
+    QuantRow row[kMaxRows];
+};
+
+struct MergeRow {
+    int64_t n;
+    int64_t word_off;
+    int64_t elem_off;    // offset of the tensor within the merged output
+    int64_t chunk_begin;
+    int vec;
+};
+
+struct MergeTable {
+    int T;
+    int W;
+    int64_t total_chunks;
+    const uint32_t *bucket[QGA_MAX_WORKERS];
+    MergeRow row[kMaxRows];
+};
+
+// Largest t with chunk_begin[t] <= chunk: the tensor owning `chunk` (a
+// tensor with no chunks shares its first-chunk number with the next one and
+// is never chosen).
+template <typename Table>
+__device__ __forceinline__ int owner_row(const Table &tab, int64_t chunk)
+{
+    int lo = 0, hi = tab.T - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (tab.row[mid].chunk_begin <= chunk)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    return lo;
+}
+
+template <typename G>
+__global__ void __launch_bounds__(kThreads)
+    quantize_2bit_bucket_kernel(const __grid_constant__ QuantTable tab, uint32_t *__restrict__ compr)
+{
+    const int lane = threadIdx.x & (kWarp - 1);
+    const int warp = threadIdx.x >> 5;
+    for (int64_t chunk = blockIdx.x; chunk < tab.total_chunks; chunk += gridDim.x) {
+        const QuantRow &row = tab.row[owner_row(tab, chunk)];
+        const int64_t c = chunk - row.chunk_begin;
+        uint32_t *rec = compr + row.word_off;
+        if (c == 0 && threadIdx.x == 0) {
+            rec[0] = bits_from_f32(row.neg);
+            rec[1] = bits_from_f32(row.pos);
+            rec[2] = bits_from_f32(__ll2float_rn(row.n));
+        }
+        const int64_t tiles = (row.n + kTileElems - 1) / kTileElems;
+        const int64_t t_end = min((c + 1) * kChunkTiles, tiles);
+        const G *grad = static_cast<const G *>(row.grad);
+        if (row.vec) {
+            for (int64_t t = c * kChunkTiles + warp; t < t_end; t += kWarpsPerBlock)
+                quantize_2bit_tile<G, true>(grad, row.residual, rec + 3, row.n, t, row.neg, row.pos, lane);
+        } else {
+            for (int64_t t = c * kChunkTiles + warp; t < t_end; t += kWarpsPerBlock)
+                quantize_2bit_tile<G, false>(grad, row.residual, rec + 3, row.n, t, row.neg, row.pos, lane);
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kThreads)
+    dequant_accumulate_2bit_bucket_kernel(const __grid_constant__ MergeTable tab, float *__restrict__ out)
+{
+    __shared__ const uint32_t *s_payload[QGA_MAX_WORKERS];
+    __shared__ float s_neg[QGA_MAX_WORKERS], s_pos[QGA_MAX_WORKERS];
+    const int lane = threadIdx.x & (kWarp - 1);
+    const int warp = threadIdx.x >> 5;
+    for (int64_t chunk = blockIdx.x; chunk < tab.total_chunks; chunk += gridDim.x) {
+        const MergeRow &row = tab.row[owner_row(tab, chunk)];
+        const int64_t c = chunk - row.chunk_begin;
+        __syncthreads(); // the previous chunk's readers of s_* are done
+        if (threadIdx.x < tab.W) {
+            const uint32_t *rec = tab.bucket[threadIdx.x] + row.word_off;
+            s_payload[threadIdx.x] = rec + 3;
+            s_neg[threadIdx.x] = f32_from_bits(rec[0]);
+            s_pos[threadIdx.x] = f32_from_bits(rec[1]);
+        }
+        __syncthreads();
+        const int64_t tiles = (row.n + kTileElems - 1) / kTileElems;
+        const int64_t t_end = min((c + 1) * kChunkTiles, tiles);
+        float *o = out + row.elem_off;
+        auto payload_of = [&](int w) { return s_payload[w]; };
+        auto neg_of = [&](int w) { return s_neg[w]; };
+        auto pos_of = [&](int w) { return s_pos[w]; };
+        if (row.vec) {
+            for (int64_t t = c * kChunkTiles + warp; t < t_end; t += kWarpsPerBlock)
+                dequant_accumulate_2bit_tile<true>(tab.W, payload_of, neg_of, pos_of, o, row.n, t, lane);
+        } else {
+            for (int64_t t = c * kChunkTiles + warp; t < t_end; t += kWarpsPerBlock)
+                dequant_accumulate_2bit_tile<false>(tab.W, payload_of, neg_of, pos_of, o, row.n, t, lane);
+        }
+    }
+}
+
+std::atomic<int> occ_qb_f32[64], occ_qb_bf16[64], occ_ab[64];
+
+int64_t chunks_of(int64_t n, bool at_least_one)
+{
+    const int64_t c = (n + kChunkElems - 1) / kChunkElems;
+    return (at_least_one && c == 0) ? 1 : c;
+}
+
+template <typename G>
+int quantize_bucket(const qga_bucket_tensor *tensors, int T, uint32_t *compr, cudaStream_t stream,
+                    std::atomic<int> *occ)
+{
+    const uintptr_t gal = GradLoad<G>::kVecAlign;
+    // validate everything before the first launch
+    for (int t = 0; t < T; ++t) {
+        const qga_bucket_tensor &d = tensors[t];
+        if (d.n < 0 || !finite_f32(d.neg_threshold) || !finite_f32(d.pos_threshold))
+            return QGA_ERR_INVALID_ARG;
+        if (d.n > 0 && (d.grad == nullptr || d.residual == nullptr || !aligned(d.grad, sizeof(G)) ||
+                        !aligned(d.residual, 4)))
+            return QGA_ERR_INVALID_ARG;
+    }
+    auto kernel = quantize_2bit_bucket_kernel<G>;
+    const int resident = resident_blocks(kernel, kThreads, occ);
+    int64_t word_off = 0;
+    for (int base = 0; base < T; base += kMaxRows) {
+        QuantTable tab;
+        tab.T = (T - base) < kMaxRows ? (T - base) : kMaxRows;
+        int64_t chunk = 0;
+        for (int i = 0; i < tab.T; ++i) {
+            const qga_bucket_tensor &d = tensors[base + i];
+            QuantRow &r = tab.row[i];
+            r.grad = d.grad;
+            r.residual = d.residual;
+            r.n = d.n;
+            r.word_off = word_off;
+            r.chunk_begin = chunk;
+            r.neg = d.neg_threshold;
+            r.pos = d.pos_threshold;
+            r.vec = aligned(d.grad, gal) && aligned(d.residual, 16);
+            chunk += chunks_of(d.n, true);
+            word_off += 3 + (d.n + 15) / 16;
+        }
+        tab.total_chunks = chunk;
+        kernel<<<grid_for(chunk, resident), kThreads, 0, stream>>>(tab, compr);
+        const int st = launch_status();
+        if (st != QGA_OK)
+            return st;
+    }
+    return QGA_OK;
+}
+
+} // namespace
+} // namespace qga
+
+using namespace qga;
+
+extern "C" int64_t qga_2bit_bucket_words(const int64_t *n, int num_tensors)
+{
+    if (num_tensors < 0 || (num_tensors > 0 && n == nullptr))
+        return QGA_ERR_INVALID_ARG;
+    int64_t words = 0;
+    for (int t = 0; t < num_tensors; ++t) {
+        if (n[t] < 0)
+            return QGA_ERR_INVALID_ARG;
+        words += 3 + (n[t] + 15) / 16;
+    }
+    return words;
+}
+
+extern "C" int qga_quantize_2bit_bucket(const qga_bucket_tensor *tensors, int num_tensors,
+                                        int grad_dtype, uint32_t *compr, cudaStream_t stream)
+{
+    if (num_tensors < 0 || (num_tensors > 0 && (tensors == nullptr || compr == nullptr)))
+        return QGA_ERR_INVALID_ARG;
+    if (compr != nullptr && !aligned(compr, 4))
+        return QGA_ERR_INVALID_ARG;
+    if (grad_dtype == QGA_DTYPE_F32)
+        return quantize_bucket<float>(tensors, num_tensors, compr, stream, occ_qb_f32);
+    if (grad_dtype == QGA_DTYPE_BF16)
+        return quantize_bucket<uint16_t>(tensors, num_tensors, compr, stream, occ_qb_bf16);
+    return QGA_ERR_UNSUPPORTED;
+}
+
+extern "C" int qga_dequant_accumulate_2bit_bucket(const uint32_t *const *compr, int num_workers,
+                                                  const int64_t *n, int num_tensors, float *out,
+                                                  cudaStream_t stream)
+{
+    if (compr == nullptr || num_workers < 1 || num_workers > QGA_MAX_WORKERS || num_tensors < 0 ||
+        (num_tensors > 0 && n == nullptr))
+        return QGA_ERR_INVALID_ARG;
+    int64_t total = 0;
+    for (int t = 0; t < num_tensors; ++t) {
+        if (n[t] < 0)
+            return QGA_ERR_INVALID_ARG;
+        total += n[t];
+    }
+    for (int w = 0; w < num_workers; ++w)
+        if (compr[w] == nullptr || !aligned(compr[w], 4))
+            return QGA_ERR_INVALID_ARG;
+    if (total == 0)
+        return QGA_OK;
+    if (out == nullptr || !aligned(out, 4))
+        return QGA_ERR_INVALID_ARG;
+    auto kernel = dequant_accumulate_2bit_bucket_kernel;
+    const int resident = resident_blocks(kernel, kThreads, occ_ab);
+    int64_t word_off = 0, elem_off = 0;
+    for (int base = 0; base < num_tensors; base += kMaxRows) {
+        MergeTable tab;
+        tab.T = (num_tensors - base) < kMaxRows ? (num_tensors - base) : kMaxRows;
+        tab.W = num_workers;
+        for (int w = 0; w < QGA_MAX_WORKERS; ++w)
+            tab.bucket[w] = w < num_workers ? compr[w] : nullptr;
+        int64_t chunk = 0;
+        for (int i = 0; i < tab.T; ++i) {
+            MergeRow &r = tab.row[i];
+            r.n = n[base + i];
+            r.word_off = word_off;
+            r.elem_off = elem_off;
+            r.chunk_begin = chunk;
+            r.vec = aligned(out + elem_off, 16);
+            chunk += chunks_of(r.n, false);
+            word_off += 3 + (r.n + 15) / 16;
+            elem_off += r.n;
+        }
+        tab.total_chunks = chunk;
+        if (chunk == 0)
+            continue;
+        kernel<<<grid_for(chunk, resident), kThreads, 0, stream>>>(tab, out);
+        const int st = launch_status();
+        if (st != QGA_OK)
+            return st;
+    }
+    return QGA_OK;
+}

@@ -1,0 +1,386 @@
+// qga_qsgd.cu -- QSGD-MaxNorm with b-bit signed codes: the global max|g|,
+// the per-worker stochastic quantizer and the integer-sum merge.
+//
+// The gradient-compression README (vineeths96), "About The Project" and
+// "Results", names QSGDMaxNorm quantization and calls it all-reduce
+// compatible; it prints no formula.  This library's definition:
+//   s = 2^(b-1) - 1,  M = max |g| over every worker's gradient,
+//   u = Philox4x32-10 draw of the element (Salmon et al., "Parallel Random
+//       Numbers: As Easy as 1, 2, 3", SC'11), top 24 bits times 2^-24,
+//   t = ((|g| / M) * s) + u  (three binary32 operations in this order),
+//   q = sign(g) * min(floor(t), s), 0 when t is not finite,
+// packed as b-bit two's complement, 32/b per word, first element in the most
+// significant bits, after a header [M, b, n].  The merge adds the integer
+// levels of all workers and scales once by M / s, which is what lets the
+// codes be summed by an all-reduce.
+//
+// Tile geometry as in the 2-bit path: a warp owns 128 groups of 4 elements;
+// lane l handles groups l, l+32, l+64, l+96 (coalesced 128-bit loads).  One
+// Philox block (one counter) yields the 4 draws of one group.
+
+#include <float.h>
+
+#include "qga_common.cuh"
+
+namespace qga {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarpsPerBlock = kThreads / kWarp;
+constexpr int kGroupsPerLane = 4;
+constexpr int kTileGroups = kWarp * kGroupsPerLane;
+
+struct GradSet {
+    const float *g[QGA_MAX_WORKERS];
+};
+
+struct RecordSet {
+    const uint32_t *rec[QGA_MAX_WORKERS];
+};
+
+// ----------------------------------------------------------- Philox4x32-10 --
+// Ten rounds of: two 32x32 -> 64-bit products of the even counter words with
+// the round multipliers; the high halves xor the odd words and the key, the
+// low halves move to the odd slots.  The key is bumped by the Weyl constants
+// before every round but the first.
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1)
+{
+#pragma unroll
+    for (int round = 0; round < 10; ++round) {
+        if (round > 0) {
+            k0 += 0x9E3779B9u;
+            k1 += 0xBB67AE85u;
+        }
+        const uint32_t hi0 = __umulhi(0xD2511F53u, c.x);
+        const uint32_t lo0 = 0xD2511F53u * c.x;
+        const uint32_t hi1 = __umulhi(0xCD9E8D57u, c.z);
+        const uint32_t lo1 = 0xCD9E8D57u * c.z;
+        c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+    }
+    return c;
+}
+
+// Draw of an output word: its top 24 bits as a multiple of 2^-24 (exact).
+__device__ __forceinline__ float unit_draw(uint32_t x)
+{
+    return __fmul_rn(__uint2float_rn(x >> 8), 0x1p-24f);
+}
+
+template <int B> struct Levels {
+    static constexpr int s = (1 << (B - 1)) - 1;
+    static constexpr uint32_t mask = (1u << B) - 1u;
+    static constexpr int lanes_per_word = 8 / B; // 4 codes of B bits per lane
+};
+
+template <int B>
+__device__ __forceinline__ int32_t qsgd_level(float g, float M, float u)
+{
+    constexpr float s = (float)Levels<B>::s;
+    const float t = __fadd_rn(__fmul_rn(__fdiv_rn(fabsf(g), M), s), u);
+    if (!(fabsf(t) <= FLT_MAX)) // NaN or infinite
+        return 0;
+    const int32_t q = (int32_t)fminf(floorf(t), s);
+    return g < 0.0f ? -q : q;
+}
+
+// ------------------------------------------------------------------- max ----
+__global__ void __launch_bounds__(kThreads)
+    qsgd_max_kernel(const __grid_constant__ GradSet set, int W, int64_t n, float *__restrict__ M)
+{
+    __shared__ float s_part[kWarpsPerBlock];
+    const int64_t tid = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+    const int64_t nthreads = (int64_t)gridDim.x * kThreads;
+    const int64_t groups = n >> 2;
+    float m = 0.0f;
+    for (int w = 0; w < W; ++w) {
+        const float *g = set.g[w];
+        if (((uintptr_t)g & 15u) == 0) {
+            int64_t i = tid;
+            for (; i + 3 * nthreads < groups; i += 4 * nthreads) {
+                const float4 a = ld_stream_f4(g + 4 * i);
+                const float4 b = ld_stream_f4(g + 4 * (i + nthreads));
+                const float4 c = ld_stream_f4(g + 4 * (i + 2 * nthreads));
+                const float4 d = ld_stream_f4(g + 4 * (i + 3 * nthreads));
+                m = fmaxf(m, fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w))));
+                m = fmaxf(m, fmaxf(fmaxf(fabsf(b.x), fabsf(b.y)), fmaxf(fabsf(b.z), fabsf(b.w))));
+                m = fmaxf(m, fmaxf(fmaxf(fabsf(c.x), fabsf(c.y)), fmaxf(fabsf(c.z), fabsf(c.w))));
+                m = fmaxf(m, fmaxf(fmaxf(fabsf(d.x), fabsf(d.y)), fmaxf(fabsf(d.z), fabsf(d.w))));
+            }
+            for (; i < groups; i += nthreads) {
+                const float4 a = ld_stream_f4(g + 4 * i);
+                m = fmaxf(m, fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w))));
+            }
+            for (int64_t e = 4 * groups + tid; e < n; e += nthreads)
+                m = fmaxf(m, fabsf(ld_stream_f1(g + e)));
+        } else {
+            for (int64_t e = tid; e < n; e += nthreads)
+                m = fmaxf(m, fabsf(ld_stream_f1(g + e)));
+        }
+    }
+    // fmaxf drops a NaN operand, so m is never NaN
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+        m = fmaxf(m, __shfl_xor_sync(kFullMask, m, off));
+    if ((threadIdx.x & 31) == 0)
+        s_part[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float b = s_part[0];
+#pragma unroll
+        for (int i = 1; i < kWarpsPerBlock; ++i)
+            b = fmaxf(b, s_part[i]);
+        // non-negative binary32 values order like their bit patterns
+        if (b > 0.0f)
+            atomicMax(reinterpret_cast<unsigned int *>(M), __float_as_uint(b));
+    }
+}
+
+// -------------------------------------------------------------- quantize ----
+template <int B, bool kVec>
+__global__ void __launch_bounds__(kThreads)
+    qsgd_quantize_kernel(const float *__restrict__ grad, uint32_t *__restrict__ compr, int64_t n,
+                         uint32_t key0, uint32_t key1, const float *__restrict__ max_in)
+{
+    using L = Levels<B>;
+    const float M = *max_in;
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        compr[0] = bits_from_f32(M);
+        compr[1] = bits_from_f32((float)B);
+        compr[2] = bits_from_f32(__ll2float_rn(n));
+    }
+    uint32_t *payload = compr + 3;
+    const int lane = threadIdx.x & (kWarp - 1);
+    const int64_t full_groups = n >> 2;
+    const int64_t groups = (n + 3) >> 2;
+    const int64_t nwords = (n * B + 31) >> 5;
+    const int64_t tiles = (groups + kTileGroups - 1) / kTileGroups;
+    const int64_t stride = (int64_t)gridDim.x * kWarpsPerBlock;
+    for (int64_t tile = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5); tile < tiles;
+         tile += stride) {
+        const int64_t g0 = tile * kTileGroups;
+        float4 gv[kGroupsPerLane];
+#pragma unroll
+        for (int j = 0; j < kGroupsPerLane; ++j) {
+            const int64_t gi = g0 + j * kWarp + lane;
+            if (kVec && gi < full_groups) {
+                gv[j] = ld_stream_f4(grad + 4 * gi);
+            } else {
+                float t[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    t[k] = (4 * gi + k < n) ? ld_stream_f1(grad + 4 * gi + k) : 0.0f;
+                gv[j] = make_float4(t[0], t[1], t[2], t[3]);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < kGroupsPerLane; ++j) {
+            const int64_t gi = g0 + j * kWarp + lane;
+            const uint4 r = philox4x32_10(
+                make_uint4((uint32_t)gi, (uint32_t)((uint64_t)gi >> 32), 0u, 0u), key0, key1);
+            const uint32_t c0 = (uint32_t)qsgd_level<B>(gv[j].x, M, unit_draw(r.x)) & L::mask;
+            const uint32_t c1 = (uint32_t)qsgd_level<B>(gv[j].y, M, unit_draw(r.y)) & L::mask;
+            const uint32_t c2 = (uint32_t)qsgd_level<B>(gv[j].z, M, unit_draw(r.z)) & L::mask;
+            const uint32_t c3 = (uint32_t)qsgd_level<B>(gv[j].w, M, unit_draw(r.w)) & L::mask;
+            uint32_t piece = (c0 << (3 * B)) | (c1 << (2 * B)) | (c2 << B) | c3;
+            // codes of elements >= n are zero
+            const int64_t valid = n - 4 * gi;
+            if (valid < 4)
+                piece = valid <= 0 ? 0u : (piece & ~((1u << (B * (4 - (int)valid))) - 1u));
+            constexpr int LW = L::lanes_per_word;
+            uint32_t word = piece << (32 - 4 * B * (1 + (lane % LW)));
+            if (LW >= 2)
+                word |= __shfl_xor_sync(kFullMask, word, 1);
+            if (LW >= 4)
+                word |= __shfl_xor_sync(kFullMask, word, 2);
+            const int64_t wi = gi / LW;
+            if ((lane % LW) == 0 && wi < nwords)
+                st_stream_u32(payload + wi, word);
+        }
+    }
+}
+
+// ----------------------------------------------------------------- merge ----
+template <int B, bool kVec>
+__global__ void __launch_bounds__(kThreads)
+    qsgd_merge_kernel(const __grid_constant__ RecordSet set, int W, float *__restrict__ out,
+                      int64_t n)
+{
+    using L = Levels<B>;
+    __shared__ const uint32_t *s_payload[QGA_MAX_WORKERS];
+    if (threadIdx.x < W)
+        s_payload[threadIdx.x] = set.rec[threadIdx.x] + 3;
+    __syncthreads();
+    const float step = __fdiv_rn(f32_from_bits(set.rec[0][0]), (float)L::s);
+    constexpr int LW = L::lanes_per_word;
+    const int lane = threadIdx.x & (kWarp - 1);
+    const int64_t groups = (n + 3) >> 2;
+    const int64_t tiles = (groups + kTileGroups - 1) / kTileGroups;
+    const int64_t stride = (int64_t)gridDim.x * kWarpsPerBlock;
+    for (int64_t tile = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5); tile < tiles;
+         tile += stride) {
+        const int64_t g0 = tile * kTileGroups;
+        int32_t acc[kGroupsPerLane][4] = {};
+        constexpr int kBatch = 8;
+        for (int wb = 0; wb < W; wb += kBatch) {
+            uint32_t words[kBatch][kGroupsPerLane];
+#pragma unroll
+            for (int k = 0; k < kBatch; ++k)
+#pragma unroll
+                for (int j = 0; j < kGroupsPerLane; ++j) {
+                    const int64_t gi = g0 + j * kWarp + lane;
+                    words[k][j] = (wb + k < W && gi < groups) ? ld_stream_u32(s_payload[wb + k] + gi / LW)
+                                                              : 0u;
+                }
+#pragma unroll
+            for (int k = 0; k < kBatch; ++k) {
+                if (wb + k < W) { // warp-uniform
+#pragma unroll
+                    for (int j = 0; j < kGroupsPerLane; ++j) {
+                        // this group's 4B bits, moved to the top of the word
+                        const uint32_t top = words[k][j] << (4 * B * (lane % LW));
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            acc[j][e] += (int32_t)(top << (B * e)) >> (32 - B);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < kGroupsPerLane; ++j) {
+            const int64_t gi = g0 + j * kWarp + lane;
+            const float4 v = make_float4(__fmul_rn(__int2float_rn(acc[j][0]), step),
+                                         __fmul_rn(__int2float_rn(acc[j][1]), step),
+                                         __fmul_rn(__int2float_rn(acc[j][2]), step),
+                                         __fmul_rn(__int2float_rn(acc[j][3]), step));
+            if (kVec && gi < (n >> 2)) {
+                st_stream_f4(out + 4 * gi, v);
+            } else {
+                const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    if (4 * gi + k < n)
+                        st_stream_f1(out + 4 * gi + k, vv[k]);
+            }
+        }
+    }
+}
+
+std::atomic<int> occ_max[64];
+std::atomic<int> occ_q[3][2][64];
+std::atomic<int> occ_m[3][2][64];
+
+int bits_slot(int bits) { return bits == 2 ? 0 : (bits == 4 ? 1 : (bits == 8 ? 2 : -1)); }
+
+unsigned group_grid(int64_t n, int resident)
+{
+    const int64_t groups = (n + 3) >> 2;
+    const int64_t tiles = (groups + kTileGroups - 1) / kTileGroups;
+    return grid_for((tiles + kWarpsPerBlock - 1) / kWarpsPerBlock, resident);
+}
+
+template <int B>
+void launch_quantize(const float *grad, uint32_t *compr, int64_t n, uint64_t seed, const float *M,
+                     cudaStream_t stream)
+{
+    const uint32_t k0 = (uint32_t)seed, k1 = (uint32_t)(seed >> 32);
+    const int s = bits_slot(B);
+    if (aligned(grad, 16)) {
+        auto k = qsgd_quantize_kernel<B, true>;
+        k<<<group_grid(n, resident_blocks(k, kThreads, occ_q[s][0])), kThreads, 0, stream>>>(
+            grad, compr, n, k0, k1, M);
+    } else {
+        auto k = qsgd_quantize_kernel<B, false>;
+        k<<<group_grid(n, resident_blocks(k, kThreads, occ_q[s][1])), kThreads, 0, stream>>>(
+            grad, compr, n, k0, k1, M);
+    }
+}
+
+template <int B>
+void launch_merge(const RecordSet &set, int W, float *out, int64_t n, cudaStream_t stream)
+{
+    const int s = bits_slot(B);
+    if (aligned(out, 16)) {
+        auto k = qsgd_merge_kernel<B, true>;
+        k<<<group_grid(n, resident_blocks(k, kThreads, occ_m[s][0])), kThreads, 0, stream>>>(
+            set, W, out, n);
+    } else {
+        auto k = qsgd_merge_kernel<B, false>;
+        k<<<group_grid(n, resident_blocks(k, kThreads, occ_m[s][1])), kThreads, 0, stream>>>(
+            set, W, out, n);
+    }
+}
+
+} // namespace
+} // namespace qga
+
+using namespace qga;
+
+extern "C" int64_t qga_qsgd_words(int64_t n, int bits)
+{
+    if (n < 0 || bits_slot(bits) < 0)
+        return n < 0 ? QGA_ERR_INVALID_ARG : QGA_ERR_UNSUPPORTED;
+    return 3 + (n * bits + 31) / 32;
+}
+
+extern "C" int qga_qsgd_mn_max(const float *const *grad, int num_workers, int64_t n,
+                               float *max_out, cudaStream_t stream)
+{
+    if (grad == nullptr || num_workers < 1 || num_workers > QGA_MAX_WORKERS || n < 0 ||
+        max_out == nullptr || !aligned(max_out, 4))
+        return QGA_ERR_INVALID_ARG;
+    GradSet set{};
+    for (int w = 0; w < num_workers; ++w) {
+        if (n > 0 && (grad[w] == nullptr || !aligned(grad[w], 4)))
+            return QGA_ERR_INVALID_ARG;
+        set.g[w] = grad[w];
+    }
+    int st = cuda_status(cudaMemsetAsync(max_out, 0, sizeof(float), stream));
+    if (st != QGA_OK || n == 0)
+        return st;
+    const int64_t groups = (n + 3) >> 2;
+    const int resident = resident_blocks(qsgd_max_kernel, kThreads, occ_max);
+    qsgd_max_kernel<<<grid_for((groups + kThreads - 1) / kThreads, resident), kThreads, 0, stream>>>(
+        set, num_workers, n, max_out);
+    return launch_status();
+}
+
+extern "C" int qga_qsgd_mn_quantize(const float *grad, uint32_t *compr, int64_t n, int bits,
+                                    uint64_t seed, const float *max_in, cudaStream_t stream)
+{
+    if (n < 0 || compr == nullptr || !aligned(compr, 4) || max_in == nullptr || !aligned(max_in, 4))
+        return QGA_ERR_INVALID_ARG;
+    if (n > 0 && (grad == nullptr || !aligned(grad, 4)))
+        return QGA_ERR_INVALID_ARG;
+    switch (bits) {
+    case 2: launch_quantize<2>(grad, compr, n, seed, max_in, stream); break;
+    case 4: launch_quantize<4>(grad, compr, n, seed, max_in, stream); break;
+    case 8: launch_quantize<8>(grad, compr, n, seed, max_in, stream); break;
+    default: return QGA_ERR_UNSUPPORTED;
+    }
+    return launch_status();
+}
+
+extern "C" int qga_qsgd_mn_dequant_accumulate(const uint32_t *const *compr, int num_workers,
+                                              float *out, int64_t n, int bits, cudaStream_t stream)
+{
+    if (compr == nullptr || num_workers < 1 || num_workers > QGA_MAX_WORKERS || n < 0)
+        return QGA_ERR_INVALID_ARG;
+    if (bits_slot(bits) < 0)
+        return QGA_ERR_UNSUPPORTED;
+    RecordSet set{};
+    for (int w = 0; w < num_workers; ++w) {
+        if (compr[w] == nullptr || !aligned(compr[w], 4))
+            return QGA_ERR_INVALID_ARG;
+        set.rec[w] = compr[w];
+    }
+    if (n == 0)
+        return QGA_OK;
+    if (out == nullptr || !aligned(out, 4))
+        return QGA_ERR_INVALID_ARG;
+    switch (bits) {
+    case 2: launch_merge<2>(set, num_workers, out, n, stream); break;
+    case 4: launch_merge<4>(set, num_workers, out, n, stream); break;
+    default: launch_merge<8>(set, num_workers, out, n, stream); break;
+    }
+    return launch_status();
+}

@@ -1,0 +1,191 @@
+"""GPU parity of QSGD-MaxNorm (max, b-bit quantize, integer-sum merge)
+against the CPU oracle: M exact, codes bit for bit, merged values bit for bit
+(the level sum is an integer, so the order of workers cannot matter) and
+within 1e-6 relative + 1e-7 absolute."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from gpu_util import AGG_ATOL, AGG_RTOL, DEV, f32, first_diff, offset_view, qga, same_bits_f32, u32
+
+pytestmark = pytest.mark.gpu
+
+BITS = [2, 4, 8]
+
+
+def _grads(W, n, seed, offsets=None, scale=2.0):
+    gen = torch.Generator(device=DEV)
+    gen.manual_seed(seed)
+    out = []
+    for w in range(W):
+        g = offset_view(n, torch.float32, offsets[w] if offsets else 0)
+        g.copy_(torch.randn(n, device=DEV, generator=gen) * scale)
+        out.append(g)
+    return out
+
+
+@pytest.mark.parametrize("W", [1, 3, 8, 64])
+@pytest.mark.parametrize("n", [1, 3, 17, 4097, 1_000_003])
+def test_max(W, n):
+    grads = _grads(W, n, W * 7 + n, offsets=[w % 3 for w in range(W)])
+    M = torch.full((1,), -1.0, device=DEV)
+    qga().qga_qsgd_mn_max(grads, M)
+    want = oracle.qsgd_mn_max([f32(g) for g in grads])
+    assert M.item() == want
+    assert M.item() == torch.stack([g.abs().max() for g in grads]).max().item()
+
+
+def test_max_special_values():
+    g = torch.tensor([0.0, -0.0, float("nan"), -3.5, 1.0, float("nan")], device=DEV)
+    M = torch.zeros(1, device=DEV)
+    qga().qga_qsgd_mn_max([g], M)
+    assert M.item() == 3.5 == oracle.qsgd_mn_max([f32(g)])
+    z = torch.zeros(1000, device=DEV)
+    M.fill_(7.0)
+    qga().qga_qsgd_mn_max([z, z], M)
+    assert M.item() == 0.0
+
+
+@pytest.mark.parametrize("b", BITS)
+@pytest.mark.parametrize("n", [0, 1, 3, 4, 5, 15, 16, 17, 31, 33, 127, 129, 513, 4097, 65_537,
+                               (1 << 20) + 7])
+def test_quantize(b, n):
+    q = qga()
+    (g,) = _grads(1, n, 100 + n)
+    g_host = f32(g)
+    M = torch.empty(1, device=DEV)
+    if n:
+        q.qga_qsgd_mn_max([g], M)
+        M_oracle = oracle.qsgd_mn_max([g_host])
+        assert M.item() == M_oracle
+    else:
+        M.fill_(1.0)
+        M_oracle = np.float32(1.0)
+    seed = 0x1234_5678_9ABC_DEF0 + n
+    words = q.qga_qsgd_words(n, b)
+    buf = torch.full((words + 4,), -1, dtype=torch.int32, device=DEV)
+    buf[words:] = 0x5A5A5A5A
+    q.qga_qsgd_mn_quantize(g, buf[:words], b, seed, M)
+    got = u32(buf)
+    assert (got[words:] == 0x5A5A5A5A).all()
+    want = oracle.qsgd_mn_quantize(g_host, b, seed, M_oracle)
+    assert np.array_equal(got[:words], want), first_diff(got[:words], want)
+
+
+@pytest.mark.parametrize("b", BITS)
+def test_quantize_misaligned_and_special(b):
+    q = qga()
+    vals = np.array([0.0, -0.0, 50.0, -50.0, 1e-40, -1e-40, 49.999996, -0.5, 25.0, 12.5, 60.0,
+                     float("nan"), float("inf")], np.float32)
+    n = vals.size
+    g = offset_view(n, torch.float32, 1)
+    g.copy_(torch.from_numpy(vals))
+    M = torch.tensor([50.0], device=DEV)
+    words = q.qga_qsgd_words(n, b)
+    c = torch.empty(words, dtype=torch.int32, device=DEV)
+    q.qga_qsgd_mn_quantize(g, c, b, 42, M)
+    assert np.array_equal(u32(c), oracle.qsgd_mn_quantize(vals, b, 42, np.float32(50.0)))
+    # M == 0: every level is 0
+    M.zero_()
+    q.qga_qsgd_mn_quantize(g, c, b, 42, M)
+    assert np.array_equal(u32(c), oracle.qsgd_mn_quantize(vals, b, 42, np.float32(0.0)))
+    assert not u32(c)[3:].any()
+
+
+@pytest.mark.parametrize("b", BITS)
+@pytest.mark.parametrize("W", [1, 2, 8, 64])
+@pytest.mark.parametrize("n", [1, 17, 513, 65_537])
+def test_merge(b, W, n):
+    q = qga()
+    grads = _grads(W, n, 1000 * b + W + n)
+    hosts = [f32(g) for g in grads]
+    M = torch.empty(1, device=DEV)
+    q.qga_qsgd_mn_max(grads, M)
+    M_oracle = oracle.qsgd_mn_max(hosts)
+    assert M.item() == M_oracle
+    comprs, want_recs = [], []
+    for w, g in enumerate(grads):
+        c = torch.empty(q.qga_qsgd_words(n, b), dtype=torch.int32, device=DEV)
+        q.qga_qsgd_mn_quantize(g, c, b, 1234 + w, M)
+        comprs.append(c)
+        want_recs.append(oracle.qsgd_mn_quantize(hosts[w], b, 1234 + w, M_oracle))
+        assert np.array_equal(u32(c), want_recs[-1])
+    out = offset_view(n, torch.float32, n % 3, fill=float("nan"))
+    q.qga_qsgd_mn_dequant_accumulate(comprs, out, b)
+    want = oracle.qsgd_mn_dequant_accumulate(want_recs, n, b)
+    got = f32(out)
+    np.testing.assert_allclose(got, want, rtol=AGG_RTOL, atol=AGG_ATOL)
+    assert same_bits_f32(got, want), first_diff(got, want)
+
+
+def _levels_of_word(word, b):
+    per = 32 // b
+    out = []
+    for i in range(per):
+        d = (int(word) >> (32 - b * (i + 1))) & ((1 << b) - 1)
+        out.append(d - (1 << b) if d >= (1 << (b - 1)) else d)
+    return out
+
+
+def _pack_levels(levels, b):
+    """Oracle levels -> record words (test plumbing: the layout only)."""
+    per = 32 // b
+    words = []
+    for i in range(0, len(levels), per):
+        wd = 0
+        for j, lv in enumerate(levels[i:i + per]):
+            wd |= (int(lv) & ((1 << b) - 1)) << (32 - b * (j + 1))
+        words.append(wd)
+    return np.array(words, np.uint32)
+
+
+def test_qsgd_128M_eight_workers_sampled():
+    """The QSGD workload at full size (2^27 elements, 0.1% outliers of 50,
+    8 workers, seeds 1234 + w): M is exactly 50 and equals torch's max|g|;
+    for b = 2, 4, 8, sampled words decode to the oracle's levels at their
+    global element indices, and sampled merged values match the oracle."""
+    w = workloads.WORKLOADS["qsgd-128M-8w"]
+    n = w.n
+    q = qga()
+    grads = [workloads.gradient(w, k, 0, device=DEV) for k in range(w.workers)]
+    M = torch.empty(1, device=DEV)
+    q.qga_qsgd_mn_max(grads, M)
+    # the planted outliers fix M (an input-recipe value, not a GPU result)
+    Mf = np.float32(workloads.QSGD_OUTLIER_MAGNITUDE)
+    assert M.item() == Mf
+    assert M.item() == max(g.abs().max().item() for g in grads)
+    rng = np.random.default_rng(5)
+    for b in w.bits:
+        per = 32 // b
+        nwords = q.qga_qsgd_words(n, b) - 3
+        pick = np.unique(np.concatenate([[0, nwords - 1], rng.integers(0, nwords, 300)]))
+        elems = (pick[:, None] * per + np.arange(per)[None, :]).reshape(-1)
+        idx = torch.from_numpy(elems).to(DEV)
+        comprs = []
+        mini_records = []
+        for k, g in enumerate(grads):
+            c = torch.empty(q.qga_qsgd_words(n, b), dtype=torch.int32, device=DEV)
+            q.qga_qsgd_mn_quantize(g, c, b, workloads.QSGD_SEED_BASE + k, M)
+            comprs.append(c)
+            header = u32(c[:3])
+            assert np.array_equal(header, np.array([Mf, b, n], np.float32).view(np.uint32))
+            words = u32(c.index_select(0, torch.from_numpy(pick + 3).to(DEV)))
+            g_s = f32(g.index_select(0, idx))
+            got_levels = np.array([lv for wd in words for lv in _levels_of_word(wd, b)])
+            want_levels = np.array([oracle.qsgd_level(g_s[i], Mf, b, workloads.QSGD_SEED_BASE + k,
+                                                      int(e)) for i, e in enumerate(elems)])
+            assert np.array_equal(got_levels, want_levels), (b, k, first_diff(got_levels, want_levels))
+            assert np.abs(got_levels).max() <= 2 ** (b - 1) - 1
+            packed = _pack_levels(want_levels, b)
+            assert [lv for wd in packed for lv in _levels_of_word(wd, b)] == want_levels.tolist()
+            head = np.array([Mf, b, elems.size], np.float32).view(np.uint32)
+            mini_records.append(np.concatenate([head, packed]))
+        out = torch.empty(n, device=DEV)
+        q.qga_qsgd_mn_dequant_accumulate(comprs, out, b)
+        got = f32(out.index_select(0, idx))
+        want = oracle.qsgd_mn_dequant_accumulate(mini_records, elems.size, b)
+        np.testing.assert_allclose(got, want, rtol=AGG_RTOL, atol=AGG_ATOL)
+        assert same_bits_f32(got, want)
+        del comprs
