@@ -56,6 +56,8 @@ def parse_args():
     p.add_argument("--impl", choices=["qga", "reference"], default="qga")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-rows", action="store_true",
+                   help="skip the per-kernel timings of the other hot-path rows")
     # smaller cases of the same step, for profiler captures (not bench lines)
     p.add_argument("--n", type=int, default=None, help="elements per worker (default: workload n)")
     p.add_argument("--iterations", type=int, default=None, help="resident gradient sets")
@@ -313,7 +315,9 @@ def run_qga(args, rank, world, local_rank):
 
     e2e = None if args.no_e2e else run_e2e(args, w, grads[0], res, comprs, out, quant, merge,
                                            stream, world, dev)
-    del grads
+    del grads, res, comprs, out
+    torch.cuda.empty_cache()
+    rows = None if args.no_rows else time_rows(dev, stream, measured_peaks()[0])
 
     if rank != 0:
         return
@@ -349,11 +353,140 @@ def run_qga(args, rank, world, local_rank):
         "clocks": clocks,
         "csrc": csrc_hash(),
     }
+    if rows is not None:
+        line["kernels"].update(rows)
+        line["gpu_launches_rows"] = sum(r.get("launches", 0) for r in rows.values())
     if e2e is not None:
         line["e2e"] = e2e
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
     print(json.dumps(line), flush=True)
+
+
+def _time_launches(stream, fn, reps, warmup=3):
+    """Average device time of fn() (one or more kernel launches) over reps,
+    CUDA events on the launching stream."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(reps):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps * 1e-3
+
+
+def _row(seconds, elems, bytes_per_elem, peak, launches, **extra):
+    gbs = bytes_per_elem * elems / seconds / 1e9
+    d = {"us": seconds * 1e6, "gelem_s": elems / seconds / 1e9, "gb_s": gbs,
+         "bytes_per_elem": bytes_per_elem, "frac_of_peak": gbs / peak, "frac_of_8TBs": gbs / 8000.0,
+         "launches": launches}
+    d.update(extra)
+    return d
+
+
+def time_rows(dev, stream, peak, reps=20):
+    """Device time of every other row of the hot path, each on its own
+    workload at full size (inputs resident, larger than L2)."""
+    import torch
+
+    import quantized_gradient_aggregation_b200 as q
+    import workloads
+    rows = {}
+    L = q.lib()
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    vp = ctypes.c_void_p
+
+    def ok(st, name):
+        if st:
+            raise q.QGAError(st, name)
+
+    # dequantize of one VGG16-sized record
+    w = workloads.WORKLOADS[WORKLOAD]
+    n = w.n
+    g = workloads.gradient(w, 0, 0, device=dev)
+    r = torch.zeros(n, device=dev)
+    c = torch.empty(q.qga_2bit_words(n), dtype=torch.int32, device=dev)
+    q.qga_quantize_2bit(g, r, c, w.neg_thr, w.pos_thr)
+    out = torch.empty(n, device=dev)
+    t = _time_launches(stream, lambda: ok(L.qga_dequantize_2bit(vp(c.data_ptr()), vp(out.data_ptr()),
+                                                                n, sp), "dequantize"), reps)
+    rows["dequantize_2bit"] = _row(t, n, 4.25, peak, reps + 3, workload="vgg16 record, n=138,357,544")
+    del g, r, c, out
+
+    # BERT-Base bucket: quantize (bf16 grad) and 4-worker merge
+    wb = workloads.WORKLOADS["bert-bucket-4w"]
+    sizes = workloads.bert_base_sizes()
+    total = sum(sizes)
+    words = q.qga_2bit_bucket_words(sizes)
+    comprs, tables, keep = [], [], []
+    neg = pos = None
+    for k in range(wb.workers):
+        grads = workloads.bert_bucket(wb, k, 0, device=dev)
+        if neg is None:
+            neg, pos = workloads.bert_thresholds(grads)
+        res = [torch.zeros(s, device=dev) for s in sizes]
+        tables.append(q.make_bucket_table(grads, res, neg, pos))
+        keep.append((grads, res))
+        comprs.append(torch.empty(words, dtype=torch.int32, device=dev))
+    T = len(sizes)
+
+    def quant_bucket(k=0):
+        ok(L.qga_quantize_2bit_bucket(tables[k], T, q.QGA_DTYPE_BF16, vp(comprs[k].data_ptr()), sp),
+           "quantize_bucket")
+    for k in range(wb.workers):
+        quant_bucket(k)
+    t = _time_launches(stream, quant_bucket, reps)
+    rows["quantize_2bit_bucket_bf16"] = _row(t, total, 10.25, peak, reps + 3 + wb.workers,
+                                             workload="BERT-Base bucket, 197 bf16 tensors, "
+                                                      "109,480,704 elements")
+    out = torch.empty(total, device=dev)
+    arr = (ctypes.c_void_p * wb.workers)(*[cc.data_ptr() for cc in comprs])
+    pp = ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p))
+    nn = (ctypes.c_int64 * T)(*sizes)
+    t = _time_launches(stream, lambda: ok(L.qga_dequant_accumulate_2bit_bucket(
+        pp, wb.workers, nn, T, vp(out.data_ptr()), sp), "merge_bucket"), reps)
+    rows["dequant_accumulate_2bit_bucket_w4"] = _row(t, total, 0.25 * wb.workers + 4, peak, reps + 3,
+                                                     workload="BERT-Base bucket, 4 workers")
+    del keep, comprs, out, tables
+
+    # QSGD-MaxNorm: max over 8 workers, quantize per b, merge of 8
+    wq = workloads.WORKLOADS["qsgd-128M-8w"]
+    nq, Wq = wq.n, wq.workers
+    grads = [workloads.gradient(wq, k, 0, device=dev) for k in range(Wq)]
+    M = torch.empty(1, device=dev)
+    garr = (ctypes.c_void_p * Wq)(*[gg.data_ptr() for gg in grads])
+    gp = ctypes.cast(garr, ctypes.POINTER(ctypes.c_void_p))
+    t = _time_launches(stream, lambda: ok(L.qga_qsgd_mn_max(gp, Wq, nq, vp(M.data_ptr()), sp),
+                                          "qsgd_max"), reps)
+    rows["qsgd_mn_max_w8"] = _row(t, nq * Wq, 4.0, peak, reps + 3,
+                                  workload="8 x 2^27 fp32 (0.1% outliers of 50)")
+    out = torch.empty(nq, device=dev)
+    for b in wq.bits:
+        cq = [torch.empty(q.qga_qsgd_words(nq, b), dtype=torch.int32, device=dev) for _ in range(Wq)]
+
+        def quant_q(k=0, b=b, cq=cq):
+            ok(L.qga_qsgd_mn_quantize(vp(grads[k].data_ptr()), vp(cq[k].data_ptr()), nq, b,
+                                      workloads.QSGD_SEED_BASE + k, vp(M.data_ptr()), sp),
+               "qsgd_quantize")
+        for k in range(Wq):
+            quant_q(k)
+        t = _time_launches(stream, quant_q, reps)
+        rows[f"qsgd_mn_quantize_b{b}"] = _row(t, nq, 4 + b / 8, peak, reps + 3 + Wq,
+                                              workload=f"2^27 fp32, b={b}")
+        carr = (ctypes.c_void_p * Wq)(*[cc.data_ptr() for cc in cq])
+        cp = ctypes.cast(carr, ctypes.POINTER(ctypes.c_void_p))
+        t = _time_launches(stream, lambda: ok(L.qga_qsgd_mn_dequant_accumulate(
+            cp, Wq, vp(out.data_ptr()), nq, b, sp), "qsgd_merge"), reps)
+        rows[f"qsgd_mn_dequant_accumulate_b{b}_w8"] = _row(t, nq, Wq * b / 8 + 4, peak, reps + 3,
+                                                          workload=f"8 records of 2^27, b={b}")
+        del cq
+    del grads, out
+    torch.cuda.empty_cache()
+    return rows
 
 
 def run_e2e(args, w, dev_grads, res, comprs, out, quant, merge, stream, world, dev):

@@ -54,13 +54,17 @@ struct RecordSet {
     const uint32_t *rec[QGA_MAX_WORKERS];
 };
 
-template <bool kVec>
-__global__ void __launch_bounds__(kThreads)
+// kW > 0: compiled for exactly kW workers (record pointers and loop bounds
+// are constants); kW == 0: any W up to QGA_MAX_WORKERS.
+template <bool kVec, int kW>
+__global__ void __launch_bounds__(kThreads, 4)
     dequant_accumulate_2bit_kernel(const __grid_constant__ RecordSet set, int W,
                                    float *__restrict__ out, int64_t n)
 {
     __shared__ const uint32_t *s_payload[QGA_MAX_WORKERS];
     __shared__ float s_neg[QGA_MAX_WORKERS], s_pos[QGA_MAX_WORKERS];
+    __shared__ float2 s_table[QGA_MAX_WORKERS][16];
+    __shared__ float4 s_stage[kWarpsPerBlock][kStagePerWarp];
     if (threadIdx.x < W) {
         const uint32_t *r = set.rec[threadIdx.x];
         s_payload[threadIdx.x] = r + 3;
@@ -68,21 +72,63 @@ __global__ void __launch_bounds__(kThreads)
         s_pos[threadIdx.x] = f32_from_bits(r[1]);
     }
     __syncthreads();
+    for (int i = threadIdx.x; i < W * 16; i += kThreads)
+        s_table[i >> 4][i & 15] = pair_entry(i & 15, s_neg[i >> 4], s_pos[i >> 4]);
+    __syncthreads();
     const int lane = threadIdx.x & (kWarp - 1);
-    const int64_t tiles = (n + kTileElems - 1) / kTileElems;
-    for (int64_t t = first_tile(); t < tiles; t += tile_stride())
-        dequant_accumulate_2bit_tile<kVec>(
-            W, [&](int w) { return s_payload[w]; }, [&](int w) { return s_neg[w]; },
-            [&](int w) { return s_pos[w]; }, out, n, t, lane);
+    const int64_t slices = (n + kSliceElems - 1) / kSliceElems;
+    for (int64_t sl = first_tile(); sl < slices; sl += tile_stride()) {
+        if (kW > 0)
+            dequant_accumulate_2bit_slice<kVec, kW>(
+                W, [&](int w) { return set.rec[w] + 3; }, [&](int w) { return s_neg[w]; },
+                [&](int w) { return s_pos[w]; }, s_table, out, n, sl, lane, s_stage[threadIdx.x >> 5]);
+        else
+            dequant_accumulate_2bit_slice<kVec, 0>(
+                W, [&](int w) { return s_payload[w]; }, [&](int w) { return s_neg[w]; },
+                [&](int w) { return s_pos[w]; }, s_table, out, n, sl, lane, s_stage[threadIdx.x >> 5]);
+    }
 }
 
 std::atomic<int> occ_q_f32_v[64], occ_q_f32_s[64], occ_q_bf16_v[64], occ_q_bf16_s[64];
-std::atomic<int> occ_dq_v[64], occ_dq_s[64], occ_acc_v[64], occ_acc_s[64];
+std::atomic<int> occ_dq_v[64], occ_dq_s[64];
+std::atomic<int> occ_acc[2][9][64]; // [vec][kW][device]
 
-unsigned tiles_grid(int64_t n, int resident)
+unsigned tiles_grid(int64_t n, int resident, int64_t elems_per_warp = kTileElems)
 {
-    const int64_t tiles = (n + kTileElems - 1) / kTileElems;
+    const int64_t tiles = (n + elems_per_warp - 1) / elems_per_warp;
     return grid_for((tiles + kWarpsPerBlock - 1) / kWarpsPerBlock, resident);
+}
+
+template <bool kVec, int kW>
+void launch_merge_k(const RecordSet &set, int W, float *out, int64_t n, cudaStream_t stream)
+{
+    auto k = dequant_accumulate_2bit_kernel<kVec, kW>;
+    k<<<tiles_grid(n, resident_blocks(k, kThreads, occ_acc[kVec][kW]), kSliceElems), kThreads, 0,
+        stream>>>(set, W, out, n);
+}
+
+template <bool kVec>
+void launch_merge_v(const RecordSet &set, int W, float *out, int64_t n, cudaStream_t stream)
+{
+    switch (W) {
+    case 1: launch_merge_k<kVec, 1>(set, W, out, n, stream); break;
+    case 2: launch_merge_k<kVec, 2>(set, W, out, n, stream); break;
+    case 3: launch_merge_k<kVec, 3>(set, W, out, n, stream); break;
+    case 4: launch_merge_k<kVec, 4>(set, W, out, n, stream); break;
+    case 5: launch_merge_k<kVec, 5>(set, W, out, n, stream); break;
+    case 6: launch_merge_k<kVec, 6>(set, W, out, n, stream); break;
+    case 7: launch_merge_k<kVec, 7>(set, W, out, n, stream); break;
+    case 8: launch_merge_k<kVec, 8>(set, W, out, n, stream); break;
+    default: launch_merge_k<kVec, 0>(set, W, out, n, stream); break;
+    }
+}
+
+void launch_merge(const RecordSet &set, int W, float *out, int64_t n, cudaStream_t stream, bool vec)
+{
+    if (vec)
+        launch_merge_v<true>(set, W, out, n, stream);
+    else
+        launch_merge_v<false>(set, W, out, n, stream);
 }
 
 template <typename G>
@@ -168,14 +214,6 @@ extern "C" int qga_dequant_accumulate_2bit(const uint32_t *const *compr, int num
         return QGA_OK;
     if (out == nullptr || !aligned(out, 4))
         return QGA_ERR_INVALID_ARG;
-    if (aligned(out, 16)) {
-        auto k = dequant_accumulate_2bit_kernel<true>;
-        k<<<tiles_grid(n, resident_blocks(k, kThreads, occ_acc_v)), kThreads, 0, stream>>>(
-            set, num_workers, out, n);
-    } else {
-        auto k = dequant_accumulate_2bit_kernel<false>;
-        k<<<tiles_grid(n, resident_blocks(k, kThreads, occ_acc_s)), kThreads, 0, stream>>>(
-            set, num_workers, out, n);
-    }
+    launch_merge(set, num_workers, out, n, stream, aligned(out, 16));
     return launch_status();
 }

@@ -196,49 +196,141 @@ __device__ __forceinline__ void dequantize_2bit_tile(const uint32_t *__restrict_
     }
 }
 
-// Merge of W records for tile `tile`: values summed from +0 in worker order.
-//   payload_of(w) -> pointer to worker w's payload (word 3 of its record)
-//   neg_of(w), pos_of(w) -> its thresholds
-// Words of 8 workers are loaded before any is decoded, so each lane keeps 8
-// independent loads in flight.
-template <bool kVec, typename PayloadOf, typename NegOf, typename PosOf>
-__device__ __forceinline__ void dequant_accumulate_2bit_tile(int W, PayloadOf payload_of,
-                                                             NegOf neg_of, PosOf pos_of,
-                                                             float *__restrict__ out, int64_t n,
-                                                             int64_t tile, int lane)
-{
-    constexpr int kBatch = 8;
-    const int64_t nwords = (n + 15) >> 4;
-    const int64_t w_idx = tile * kTileWords + lane;
-    const bool in_range = w_idx < nwords;
-    float4 acc[kGroupsPerLane];
-#pragma unroll
-    for (int j = 0; j < kGroupsPerLane; ++j)
-        acc[j] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+// ------------------------------------------------------------------ merge --
+// Decoding the way the quantizer packs (one byte per lane, a shuffle per
+// worker) leaves the merge bound by instruction issue, far from HBM.  So
+// the merge has its own geometry: a warp owns a slice of 64 consecutive
+// words (1024 elements), lane l owns words l and 32 + l of the slice and
+// decodes all 16 codes of each itself -- one coalesced 32-bit load per lane
+// per worker, no shuffle -- keeping both words in flight together.
+//
+// Two decoders share the work so that neither execution pipe saturates:
+//   even workers: a 16-entry table per worker in shared memory maps 4 code
+//     bits (two elements) to the two values they stand for; one 64-bit
+//     shared load and one paired add (__fadd2_rn) per two elements (load
+//     / store pipe + FMA pipe);
+//   odd workers: each word becomes two bit masks (elements coded 01, coded
+//     10; 11 is in neither) and every element takes a predicated add of the
+//     threshold its code stands for (integer pipe + FMA pipe).
+// Both add exactly the oracle's value in the oracle's order: the table holds
+// the thresholds themselves, paired adds are two independent round-to-
+// nearest adds, and skipping the add of +0 for code 00 changes nothing (the
+// sum starts at +0, can never become -0 in round-to-nearest, and x + (+0) ==
+// x for every other x).
+// The 16 sums of a word are consecutive floats owned by one lane; they leave
+// through a per-warp shared-memory stage (xor-swizzled so that both the
+// 128-bit writes and the 128-bit reads are free of bank conflicts) as fully
+// coalesced 128-bit rows.
+constexpr int kMergeSlots = 2;                         // words per lane per slice
+constexpr int kSliceWords = kWarp * kMergeSlots;       // 64
+constexpr int64_t kSliceElems = kSliceWords * 16;      // 1024
+constexpr int kStagePerWarp = kSliceWords * 4;         // float4 per warp (4 KB)
+constexpr int kMergeBatch = 8;                         // workers loaded before decoding
 
-    for (int wb = 0; wb < W; wb += kBatch) {
-        uint32_t words[kBatch];
+// Stage position of chunk c (elements 4c..4c+3) of lane L's word.
+__device__ __forceinline__ int stage_slot(int L, int c) { return L * 4 + (c ^ ((L >> 1) & 3)); }
+
+// Pair table of one worker: entry e = (value of code e >> 2, value of code
+// e & 3), the first element of the pair in the high bits.
+__device__ __forceinline__ float2 pair_entry(int e, float neg, float pos)
+{
+    return make_float2(tb_value((uint32_t)e >> 2, neg, pos), tb_value((uint32_t)e & 3u, neg, pos));
+}
+
+// Merge slice `slice` of W records into out (n elements), values summed
+// from +0 in worker order 0..W-1.
+//   payload_of(w) -> worker w's payload (word 3 of its record)
+//   neg_of(w), pos_of(w) -> its thresholds
+//   table -> QGA_MAX_WORKERS x 16 pair entries (built by the caller for w < W)
+//   stage -> this warp's kStagePerWarp float4 of shared memory
+//   kW > 0: the worker count is the compile-time constant kW (W is ignored)
+// All 32 lanes must call this together (warp-uniform `slice`).
+template <bool kVec, int kW, typename PayloadOf, typename NegOf, typename PosOf>
+__device__ __forceinline__ void dequant_accumulate_2bit_slice(int W_runtime, PayloadOf payload_of,
+                                                              NegOf neg_of, PosOf pos_of,
+                                                              const float2 (*table)[16],
+                                                              float *__restrict__ out, int64_t n,
+                                                              int64_t slice, int lane,
+                                                              float4 *__restrict__ stage)
+{
+    const int W = kW > 0 ? kW : W_runtime;
+    const int64_t nwords = (n + 15) >> 4;
+    int64_t k[kMergeSlots];
+    bool ok[kMergeSlots];
 #pragma unroll
-        for (int k = 0; k < kBatch; ++k)
-            words[k] = (wb + k < W && in_range) ? ld_stream_u32(payload_of(wb + k) + w_idx) : 0u;
+    for (int s = 0; s < kMergeSlots; ++s) {
+        k[s] = slice * kSliceWords + s * kWarp + lane;
+        ok[s] = k[s] < nwords;
+    }
+    float2 acc[kMergeSlots][8];
 #pragma unroll
-        for (int k = 0; k < kBatch; ++k) {
-            if (wb + k < W) { // warp-uniform
-                const float neg = neg_of(wb + k), pos = pos_of(wb + k);
+    for (int s = 0; s < kMergeSlots; ++s)
 #pragma unroll
-                for (int j = 0; j < kGroupsPerLane; ++j) {
-                    const float4 v = tb_decode4(tb_group_byte(words[k], j, lane), neg, pos);
-                    acc[j].x = __fadd_rn(acc[j].x, v.x);
-                    acc[j].y = __fadd_rn(acc[j].y, v.y);
-                    acc[j].z = __fadd_rn(acc[j].z, v.z);
-                    acc[j].w = __fadd_rn(acc[j].w, v.w);
+        for (int p = 0; p < 8; ++p)
+            acc[s][p] = make_float2(0.0f, 0.0f);
+
+    for (int wb = 0; wb < W; wb += kMergeBatch) {
+        uint32_t words[kMergeSlots][kMergeBatch];
+#pragma unroll
+        for (int i = 0; i < kMergeBatch; ++i)
+#pragma unroll
+            for (int s = 0; s < kMergeSlots; ++s)
+                words[s][i] = (ok[s] && wb + i < W) ? ld_stream_u32(payload_of(wb + i) + k[s]) : 0u;
+#pragma unroll
+        for (int i = 0; i < kMergeBatch; ++i) {
+            if (wb + i >= W) // warp-uniform
+                break;
+            if ((i & 1) == 0) {
+                const char *tb = reinterpret_cast<const char *>(table[wb + i]);
+#pragma unroll
+                for (int s = 0; s < kMergeSlots; ++s)
+#pragma unroll
+                    for (int p = 0; p < 8; ++p) {
+                        // 4 code bits of elements 2p, 2p+1, times the 8-byte entry size
+                        const int sh = 25 - 4 * p;
+                        const uint32_t off =
+                            (sh >= 0 ? (words[s][i] >> sh) : (words[s][i] << (-sh))) & 0x78u;
+                        acc[s][p] = __fadd2_rn(acc[s][p], *reinterpret_cast<const float2 *>(tb + off));
+                    }
+            } else {
+                const float neg = neg_of(wb + i), pos = pos_of(wb + i);
+#pragma unroll
+                for (int s = 0; s < kMergeSlots; ++s) {
+                    const uint32_t lo = words[s][i] & 0x55555555u;
+                    const uint32_t hi = (words[s][i] >> 1) & 0x55555555u;
+                    const uint32_t is01 = lo & ~hi, is10 = hi & ~lo;
+#pragma unroll
+                    for (int p = 0; p < 16; ++p) {
+                        const uint32_t bit = 1u << (30 - 2 * p);
+                        float &a = (p & 1) ? acc[s][p >> 1].y : acc[s][p >> 1].x;
+                        if (is01 & bit)
+                            a = __fadd_rn(a, pos);
+                        if (is10 & bit)
+                            a = __fadd_rn(a, neg);
+                    }
                 }
             }
         }
     }
+
+    const int f = (lane >> 1) & 3;
 #pragma unroll
-    for (int j = 0; j < kGroupsPerLane; ++j)
-        store_group<kVec>(out, n, tile * kTileGroups + j * kWarp + lane, acc[j]);
+    for (int s = 0; s < kMergeSlots; ++s)
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+            stage[s * (kWarp * 4) + lane * 4 + (c ^ f)] =
+                make_float4(acc[s][2 * c].x, acc[s][2 * c].y, acc[s][2 * c + 1].x, acc[s][2 * c + 1].y);
+    __syncwarp();
+#pragma unroll
+    for (int s = 0; s < kMergeSlots; ++s) {
+        const int64_t g0 = (slice * kSliceWords + s * kWarp) * 4; // first group of this slot
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int q = j * kWarp + lane;
+            store_group<kVec>(out, n, g0 + q, stage[s * (kWarp * 4) + stage_slot(q >> 2, q & 3)]);
+        }
+    }
+    __syncwarp();
 }
 
 } // namespace qga

@@ -103,11 +103,14 @@ __global__ void __launch_bounds__(kThreads)
     }
 }
 
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 3)
     dequant_accumulate_2bit_bucket_kernel(const __grid_constant__ MergeTable tab, float *__restrict__ out)
 {
     __shared__ const uint32_t *s_payload[QGA_MAX_WORKERS];
     __shared__ float s_neg[QGA_MAX_WORKERS], s_pos[QGA_MAX_WORKERS];
+    __shared__ float2 s_table[QGA_MAX_WORKERS][16];
+    __shared__ float4 s_stage[kWarpsPerBlock][kStagePerWarp];
+    constexpr int64_t kChunkSlices = kChunkElems / kSliceElems;
     const int lane = threadIdx.x & (kWarp - 1);
     const int warp = threadIdx.x >> 5;
     for (int64_t chunk = blockIdx.x; chunk < tab.total_chunks; chunk += gridDim.x) {
@@ -121,18 +124,24 @@ __global__ void __launch_bounds__(kThreads)
             s_pos[threadIdx.x] = f32_from_bits(rec[1]);
         }
         __syncthreads();
-        const int64_t tiles = (row.n + kTileElems - 1) / kTileElems;
-        const int64_t t_end = min((c + 1) * kChunkTiles, tiles);
+        for (int i = threadIdx.x; i < tab.W * 16; i += kThreads)
+            s_table[i >> 4][i & 15] = pair_entry(i & 15, s_neg[i >> 4], s_pos[i >> 4]);
+        __syncthreads();
+        const int64_t slices = (row.n + kSliceElems - 1) / kSliceElems;
+        const int64_t s_end = min((c + 1) * kChunkSlices, slices);
         float *o = out + row.elem_off;
         auto payload_of = [&](int w) { return s_payload[w]; };
         auto neg_of = [&](int w) { return s_neg[w]; };
         auto pos_of = [&](int w) { return s_pos[w]; };
+        float4 *stage = s_stage[warp];
         if (row.vec) {
-            for (int64_t t = c * kChunkTiles + warp; t < t_end; t += kWarpsPerBlock)
-                dequant_accumulate_2bit_tile<true>(tab.W, payload_of, neg_of, pos_of, o, row.n, t, lane);
+            for (int64_t sl = c * kChunkSlices + warp; sl < s_end; sl += kWarpsPerBlock)
+                dequant_accumulate_2bit_slice<true, 0>(tab.W, payload_of, neg_of, pos_of, s_table, o, row.n, sl,
+                                                    lane, stage);
         } else {
-            for (int64_t t = c * kChunkTiles + warp; t < t_end; t += kWarpsPerBlock)
-                dequant_accumulate_2bit_tile<false>(tab.W, payload_of, neg_of, pos_of, o, row.n, t, lane);
+            for (int64_t sl = c * kChunkSlices + warp; sl < s_end; sl += kWarpsPerBlock)
+                dequant_accumulate_2bit_slice<false, 0>(tab.W, payload_of, neg_of, pos_of, s_table, o, row.n, sl,
+                                                     lane, stage);
         }
     }
 }
