@@ -33,7 +33,8 @@ __global__ void __launch_bounds__(kThreads)
         compr[2] = bits_from_f32(__ll2float_rn(n));
     }
     const int lane = threadIdx.x & (kWarp - 1);
-    const int64_t tiles = (n + kTileElems - 1) / kTileElems;
+    constexpr int64_t kElems = quantize_tile_elems<G>();
+    const int64_t tiles = (n + kElems - 1) / kElems;
     for (int64_t t = first_tile(); t < tiles; t += tile_stride())
         quantize_2bit_tile<G, kVec>(grad, residual, compr + 3, n, t, neg, pos, lane);
 }
@@ -141,13 +142,14 @@ int launch_quantize(const G *grad, float *residual, uint32_t *compr, int64_t n, 
                   !aligned(residual, 4)))
         return QGA_ERR_INVALID_ARG;
     const bool vec = aligned(grad, GradLoad<G>::kVecAlign) && aligned(residual, 16);
+    constexpr int64_t kElems = quantize_tile_elems<G>();
     if (vec) {
         auto k = quantize_2bit_kernel<G, true>;
-        k<<<tiles_grid(n, resident_blocks(k, kThreads, occ_v)), kThreads, 0, stream>>>(
+        k<<<tiles_grid(n, resident_blocks(k, kThreads, occ_v), kElems), kThreads, 0, stream>>>(
             grad, residual, compr, n, neg, pos);
     } else {
         auto k = quantize_2bit_kernel<G, false>;
-        k<<<tiles_grid(n, resident_blocks(k, kThreads, occ_s)), kThreads, 0, stream>>>(
+        k<<<tiles_grid(n, resident_blocks(k, kThreads, occ_s), kElems), kThreads, 0, stream>>>(
             grad, residual, compr, n, neg, pos);
     }
     return launch_status();

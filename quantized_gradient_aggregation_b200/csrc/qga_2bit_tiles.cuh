@@ -8,20 +8,22 @@
 // thresholds) and "Format of compressed gradient" (16 codes per 32-bit word,
 // the first element in the two most significant bits).
 //
-// Tile geometry.  One warp owns a tile of 512 consecutive elements = 128
-// groups of 4 = 32 packed words.  Lane l handles groups l, l+32, l+64, l+96,
-// so every load or store instruction of the warp touches 512 contiguous
-// bytes of fp32 (fully coalesced 128-bit accesses).  A group's 4 codes form
-// one byte of its word; the 4 lanes sharing a word combine their bytes with
-// two xor-shuffles (no shared memory, so no bank conflicts), and the first
-// of them stores the word.
+// Tile geometry.  One warp owns a tile of consecutive elements in groups of
+// 4: 128 groups (512 elements, 32 packed words) for an fp32 gradient, 256
+// groups (1024 elements) for a bfloat16 one, whose narrower gradient loads
+// need more groups per lane to keep as many bytes in flight.  Lane l handles
+// groups l, l+32, l+64, ..., so every load or store instruction of the warp
+// touches contiguous bytes (fully coalesced vector accesses).  A group's 4
+// codes form one byte of its word; the 4 lanes sharing a word combine their
+// bytes with two xor-shuffles (no shared memory, so no bank conflicts), and
+// the first of them stores the word.
 #pragma once
 
 #include "qga_common.cuh"
 
 namespace qga {
 
-constexpr int kGroupsPerLane = 4;
+constexpr int kGroupsPerLane = 4;                   // fp32 tiles; see GradLoad::kGroups
 constexpr int kTileGroups = kWarp * kGroupsPerLane; // 128 groups of 4 elements
 constexpr int kTileElems = kTileGroups * 4;         // 512 elements
 constexpr int kTileWords = kTileElems / 16;         // 32 words
@@ -49,34 +51,44 @@ __device__ __forceinline__ uint32_t tb_step(float g, float &r, float neg, float 
     return c;
 }
 
-// Gradient access by element type: fp32, or bfloat16 bit patterns.
+// Gradient access by element type: fp32, or bfloat16 bit patterns.  A
+// group is loaded raw (one vector load) and widened to fp32 when it is used.
 template <typename G> struct GradLoad;
 
 template <> struct GradLoad<float> {
     static constexpr uintptr_t kVecAlign = 16;
-    static __device__ __forceinline__ float4 group(const float *g, int64_t gi)
-    {
-        return ld_stream_f4(g + 4 * gi);
-    }
-    static __device__ __forceinline__ float one(const float *g, int64_t e)
-    {
-        return ld_stream_f1(g + e);
-    }
+    static constexpr int kGroups = 4; // groups per lane per tile
+    using Raw = float4;
+    static __device__ __forceinline__ Raw raw(const float *g, int64_t gi) { return ld_stream_f4(g + 4 * gi); }
+    static __device__ __forceinline__ float4 widen(Raw v) { return v; }
+    static __device__ __forceinline__ Raw pack(const float t[4]) { return make_float4(t[0], t[1], t[2], t[3]); }
+    static __device__ __forceinline__ float one(const float *g, int64_t e) { return ld_stream_f1(g + e); }
 };
 
 template <> struct GradLoad<uint16_t> {
     static constexpr uintptr_t kVecAlign = 8;
-    static __device__ __forceinline__ float4 group(const uint16_t *g, int64_t gi)
+    static constexpr int kGroups = 8;
+    using Raw = uint2; // 4 bfloat16, element 0 in the low half of .x (little endian)
+    static __device__ __forceinline__ Raw raw(const uint16_t *g, int64_t gi) { return ld_stream_u2(g + 4 * gi); }
+    static __device__ __forceinline__ float4 widen(Raw v)
     {
-        const uint2 v = ld_stream_u2(g + 4 * gi); // little endian: element 0 in v.x low half
         return make_float4(widen_bf16(v.x & 0xffffu), widen_bf16(v.x >> 16),
                            widen_bf16(v.y & 0xffffu), widen_bf16(v.y >> 16));
+    }
+    static __device__ __forceinline__ Raw pack(const float t[4])
+    {
+        // t holds widened bfloat16 values: their high halves are the originals
+        return make_uint2((__float_as_uint(t[0]) >> 16) | (__float_as_uint(t[1]) & 0xffff0000u),
+                          (__float_as_uint(t[2]) >> 16) | (__float_as_uint(t[3]) & 0xffff0000u));
     }
     static __device__ __forceinline__ float one(const uint16_t *g, int64_t e)
     {
         return widen_bf16(ld_stream_u16(g + e));
     }
 };
+
+// Elements of one quantize tile for gradient type G.
+template <typename G> __host__ __device__ constexpr int64_t quantize_tile_elems() { return (int64_t)kWarp * GradLoad<G>::kGroups * 4; }
 
 // Codes of elements at or beyond n are forced to 00: keep the top 2*valid
 // bits of a group's byte.
@@ -95,38 +107,42 @@ __device__ __forceinline__ void quantize_2bit_tile(const G *__restrict__ grad,
                                                    uint32_t *__restrict__ payload, int64_t n,
                                                    int64_t tile, float neg, float pos, int lane)
 {
+    using GL = GradLoad<G>;
+    constexpr int kG = GL::kGroups;
     const int64_t full_groups = n >> 2;
     const int64_t nwords = (n + 15) >> 4;
-    const int64_t g0 = tile * kTileGroups;
+    const int64_t g0 = tile * (kWarp * kG);
 
-    float4 gv[kGroupsPerLane], rv[kGroupsPerLane];
+    typename GL::Raw gv[kG];
+    float4 rv[kG];
 #pragma unroll
-    for (int j = 0; j < kGroupsPerLane; ++j) {
+    for (int j = 0; j < kG; ++j) {
         const int64_t gi = g0 + j * kWarp + lane;
         if (kVec && gi < full_groups) {
-            gv[j] = GradLoad<G>::group(grad, gi);
+            gv[j] = GL::raw(grad, gi);
             rv[j] = ld_stream_f4(residual + 4 * gi);
         } else {
             float tg[4], tr[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 const int64_t e = 4 * gi + k;
-                tg[k] = e < n ? GradLoad<G>::one(grad, e) : 0.0f;
+                tg[k] = e < n ? GL::one(grad, e) : 0.0f;
                 tr[k] = e < n ? ld_stream_f1(residual + e) : 0.0f;
             }
-            gv[j] = make_float4(tg[0], tg[1], tg[2], tg[3]);
+            gv[j] = GL::pack(tg);
             rv[j] = make_float4(tr[0], tr[1], tr[2], tr[3]);
         }
     }
 
 #pragma unroll
-    for (int j = 0; j < kGroupsPerLane; ++j) {
+    for (int j = 0; j < kG; ++j) {
         const int64_t gi = g0 + j * kWarp + lane;
+        const float4 g = GL::widen(gv[j]);
         float4 r = rv[j];
-        const uint32_t c0 = tb_step(gv[j].x, r.x, neg, pos);
-        const uint32_t c1 = tb_step(gv[j].y, r.y, neg, pos);
-        const uint32_t c2 = tb_step(gv[j].z, r.z, neg, pos);
-        const uint32_t c3 = tb_step(gv[j].w, r.w, neg, pos);
+        const uint32_t c0 = tb_step(g.x, r.x, neg, pos);
+        const uint32_t c1 = tb_step(g.y, r.y, neg, pos);
+        const uint32_t c2 = tb_step(g.z, r.z, neg, pos);
+        const uint32_t c3 = tb_step(g.w, r.w, neg, pos);
         uint32_t byte = (c0 << 6) | (c1 << 4) | (c2 << 2) | c3;
         if (kVec && gi < full_groups) {
             st_stream_f4(residual + 4 * gi, r);

@@ -22,8 +22,7 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarpsPerBlock = kThreads / kWarp;
-constexpr int kChunkTiles = 16;
-constexpr int64_t kChunkElems = (int64_t)kChunkTiles * kTileElems;
+constexpr int64_t kChunkElems = 8192; // a whole number of quantize tiles and merge slices
 constexpr int kMaxRows = 256;
 
 struct QuantRow {
@@ -75,8 +74,10 @@ __device__ __forceinline__ int owner_row(const Table &tab, int64_t chunk)
     return lo;
 }
 
-template <typename G>
-__global__ void __launch_bounds__(kThreads)
+// kAllVec: every row of the table is aligned for vector access (the common
+// case; only the vector path is compiled in, which keeps registers low).
+template <typename G, bool kAllVec>
+__global__ void __launch_bounds__(kThreads, 3)
     quantize_2bit_bucket_kernel(const __grid_constant__ QuantTable tab, uint32_t *__restrict__ compr)
 {
     const int lane = threadIdx.x & (kWarp - 1);
@@ -90,10 +91,12 @@ __global__ void __launch_bounds__(kThreads)
             rec[1] = bits_from_f32(row.pos);
             rec[2] = bits_from_f32(__ll2float_rn(row.n));
         }
-        const int64_t tiles = (row.n + kTileElems - 1) / kTileElems;
+        constexpr int64_t kTile = quantize_tile_elems<G>();
+        constexpr int64_t kChunkTiles = kChunkElems / kTile;
+        const int64_t tiles = (row.n + kTile - 1) / kTile;
         const int64_t t_end = min((c + 1) * kChunkTiles, tiles);
         const G *grad = static_cast<const G *>(row.grad);
-        if (row.vec) {
+        if (kAllVec || row.vec) {
             for (int64_t t = c * kChunkTiles + warp; t < t_end; t += kWarpsPerBlock)
                 quantize_2bit_tile<G, true>(grad, row.residual, rec + 3, row.n, t, row.neg, row.pos, lane);
         } else {
@@ -103,6 +106,8 @@ __global__ void __launch_bounds__(kThreads)
     }
 }
 
+// kW > 0: compiled for exactly kW workers; kW == 0: any W up to QGA_MAX_WORKERS.
+template <int kW>
 __global__ void __launch_bounds__(kThreads, 3)
     dequant_accumulate_2bit_bucket_kernel(const __grid_constant__ MergeTable tab, float *__restrict__ out)
 {
@@ -136,17 +141,40 @@ __global__ void __launch_bounds__(kThreads, 3)
         float4 *stage = s_stage[warp];
         if (row.vec) {
             for (int64_t sl = c * kChunkSlices + warp; sl < s_end; sl += kWarpsPerBlock)
-                dequant_accumulate_2bit_slice<true, 0>(tab.W, payload_of, neg_of, pos_of, s_table, o, row.n, sl,
+                dequant_accumulate_2bit_slice<true, kW>(tab.W, payload_of, neg_of, pos_of, s_table, o, row.n, sl,
                                                     lane, stage);
         } else {
             for (int64_t sl = c * kChunkSlices + warp; sl < s_end; sl += kWarpsPerBlock)
-                dequant_accumulate_2bit_slice<false, 0>(tab.W, payload_of, neg_of, pos_of, s_table, o, row.n, sl,
+                dequant_accumulate_2bit_slice<false, kW>(tab.W, payload_of, neg_of, pos_of, s_table, o, row.n, sl,
                                                      lane, stage);
         }
     }
 }
 
-std::atomic<int> occ_qb_f32[64], occ_qb_bf16[64], occ_ab[64];
+std::atomic<int> occ_qb_f32[2][64], occ_qb_bf16[2][64], occ_ab[9][64];
+
+template <int kW>
+void launch_bucket_merge(const MergeTable &tab, float *out, cudaStream_t stream)
+{
+    auto kernel = dequant_accumulate_2bit_bucket_kernel<kW>;
+    const int resident = resident_blocks(kernel, kThreads, occ_ab[kW]);
+    kernel<<<grid_for(tab.total_chunks, resident), kThreads, 0, stream>>>(tab, out);
+}
+
+void launch_bucket_merge_any(const MergeTable &tab, float *out, cudaStream_t stream)
+{
+    switch (tab.W) {
+    case 1: launch_bucket_merge<1>(tab, out, stream); break;
+    case 2: launch_bucket_merge<2>(tab, out, stream); break;
+    case 3: launch_bucket_merge<3>(tab, out, stream); break;
+    case 4: launch_bucket_merge<4>(tab, out, stream); break;
+    case 5: launch_bucket_merge<5>(tab, out, stream); break;
+    case 6: launch_bucket_merge<6>(tab, out, stream); break;
+    case 7: launch_bucket_merge<7>(tab, out, stream); break;
+    case 8: launch_bucket_merge<8>(tab, out, stream); break;
+    default: launch_bucket_merge<0>(tab, out, stream); break;
+    }
+}
 
 int64_t chunks_of(int64_t n, bool at_least_one)
 {
@@ -156,7 +184,7 @@ int64_t chunks_of(int64_t n, bool at_least_one)
 
 template <typename G>
 int quantize_bucket(const qga_bucket_tensor *tensors, int T, uint32_t *compr, cudaStream_t stream,
-                    std::atomic<int> *occ)
+                    std::atomic<int> (*occ)[64])
 {
     const uintptr_t gal = GradLoad<G>::kVecAlign;
     // validate everything before the first launch
@@ -168,8 +196,6 @@ int quantize_bucket(const qga_bucket_tensor *tensors, int T, uint32_t *compr, cu
                         !aligned(d.residual, 4)))
             return QGA_ERR_INVALID_ARG;
     }
-    auto kernel = quantize_2bit_bucket_kernel<G>;
-    const int resident = resident_blocks(kernel, kThreads, occ);
     int64_t word_off = 0;
     for (int base = 0; base < T; base += kMaxRows) {
         QuantTable tab;
@@ -190,7 +216,18 @@ int quantize_bucket(const qga_bucket_tensor *tensors, int T, uint32_t *compr, cu
             word_off += 3 + (d.n + 15) / 16;
         }
         tab.total_chunks = chunk;
-        kernel<<<grid_for(chunk, resident), kThreads, 0, stream>>>(tab, compr);
+        bool all_vec = true;
+        for (int i = 0; i < tab.T; ++i)
+            all_vec = all_vec && tab.row[i].vec;
+        if (all_vec) {
+            auto kernel = quantize_2bit_bucket_kernel<G, true>;
+            kernel<<<grid_for(chunk, resident_blocks(kernel, kThreads, occ[1])), kThreads, 0, stream>>>(
+                tab, compr);
+        } else {
+            auto kernel = quantize_2bit_bucket_kernel<G, false>;
+            kernel<<<grid_for(chunk, resident_blocks(kernel, kThreads, occ[0])), kThreads, 0, stream>>>(
+                tab, compr);
+        }
         const int st = launch_status();
         if (st != QGA_OK)
             return st;
@@ -250,8 +287,6 @@ extern "C" int qga_dequant_accumulate_2bit_bucket(const uint32_t *const *compr, 
         return QGA_OK;
     if (out == nullptr || !aligned(out, 4))
         return QGA_ERR_INVALID_ARG;
-    auto kernel = dequant_accumulate_2bit_bucket_kernel;
-    const int resident = resident_blocks(kernel, kThreads, occ_ab);
     int64_t word_off = 0, elem_off = 0;
     for (int base = 0; base < num_tensors; base += kMaxRows) {
         MergeTable tab;
@@ -274,7 +309,7 @@ extern "C" int qga_dequant_accumulate_2bit_bucket(const uint32_t *const *compr, 
         tab.total_chunks = chunk;
         if (chunk == 0)
             continue;
-        kernel<<<grid_for(chunk, resident), kThreads, 0, stream>>>(tab, out);
+        launch_bucket_merge_any(tab, out, stream);
         const int st = launch_status();
         if (st != QGA_OK)
             return st;
