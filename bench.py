@@ -95,6 +95,26 @@ def workload_config(w, n_gpus):
     }
 
 
+# ------------------------------------------------------------- ranks ----
+
+def max_over_ranks(values, world, device="cpu"):
+    """Elementwise max of per-rank timings over all ranks (the slowest rank
+    sets the job's time).  Every rank must call it, in the same order."""
+    if world <= 1:
+        return [float(v) for v in values]
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_gelem_per_s(world, workers, n, steps, ms):
+    """Whole-job throughput: gradient elements of every simulated worker on
+    every rank, over the slowest rank's time."""
+    return world * workers * n * steps / (ms * 1e-3) / 1e9
+
+
 # ------------------------------------------------------------ clocks ----
 
 class ClockSampler:
@@ -308,10 +328,7 @@ def run_qga(args, rank, world, local_rank):
     total_ms = start.elapsed_time(end)
     quant_ms = statistics.fmean(a.elapsed_time(b) for a, b in q_ev)
     merge_ms = statistics.fmean(a.elapsed_time(b) for a, b in m_ev)
-    t = torch.tensor([total_ms, quant_ms, merge_ms], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, quant_ms, merge_ms = t.tolist()
+    total_ms, quant_ms, merge_ms = max_over_ranks([total_ms, quant_ms, merge_ms], world, dev)
 
     e2e = None if args.no_e2e else run_e2e(args, w, grads[0], res, comprs, out, quant, merge,
                                            stream, world, dev)
@@ -327,7 +344,7 @@ def run_qga(args, rank, world, local_rank):
     traffic_per_elem = MEASURED_TRAFFIC.get(csrc_hash())
     line = {
         "metric": METRIC,
-        "value": world * W * n * K / (total_ms * 1e-3) / 1e9,
+        "value": job_gelem_per_s(world, W, n, K, total_ms),
         "unit": "Gelem/s",
         "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": total_ms / K,
@@ -519,12 +536,8 @@ def run_e2e(args, w, dev_grads, res, comprs, out, quant, merge, stream, world, d
         step()
     b.record(stream)
     torch.cuda.synchronize()
-    ms = a.elapsed_time(b)
-    t = torch.tensor([ms], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms = t.item()
-    return {"value": world * W * n * K / (ms * 1e-3) / 1e9, "unit": "Gelem/s",
+    (ms,) = max_over_ranks([a.elapsed_time(b)], world, dev)
+    return {"value": job_gelem_per_s(world, W, n, K, ms), "unit": "Gelem/s",
             "h2d_bytes_per_step": W * n * 4, "d2h_bytes_per_step": n * 4, "steps": K,
             "path": "pinned host gradients -> cudaMemcpyAsync -> qga_quantize_2bit x8 -> "
                     "qga_dequant_accumulate_2bit -> pinned host aggregate"}
