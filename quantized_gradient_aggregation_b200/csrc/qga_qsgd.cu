@@ -72,8 +72,9 @@ template <int B> struct Levels {
     static constexpr int lanes_per_word = 8 / B; // 4 codes of B bits per lane
 };
 
+// The level by the definition's three operations, in their order.
 template <int B>
-__device__ __forceinline__ int32_t qsgd_level(float g, float M, float u)
+__device__ __forceinline__ int32_t qsgd_level_exact(float g, float M, float u)
 {
     constexpr float s = (float)Levels<B>::s;
     const float t = __fadd_rn(__fmul_rn(__fdiv_rn(fabsf(g), M), s), u);
@@ -81,6 +82,30 @@ __device__ __forceinline__ int32_t qsgd_level(float g, float M, float u)
         return 0;
     const int32_t q = (int32_t)fminf(floorf(t), s);
     return g < 0.0f ? -q : q;
+}
+
+// The same level with one multiply instead of the division, for a finite
+// positive M, and k = fl(s / M).  Only floor(t) matters, so: t' = fl(fl(|g| k)
+// + u) is within 2^-15 of the definition's t whenever t' < s + 1 (each of the
+// two is within 1.9e-5 of the exact real |g| s / M + u: two relative
+// roundings of at most 2^-24 on a value below 128, plus half an ulp below
+// 128), and any t' >= s + 1 caps both to s.  So wherever t' is at least
+// 2^-14 away from an integer, floor(t') == floor(t); otherwise (or if t' is
+// not finite) the exact sequence decides.  Results are identical to
+// qsgd_level_exact for every input.
+template <int B>
+__device__ __forceinline__ int32_t qsgd_level(float g, float M, float k, float u)
+{
+    constexpr float s = (float)Levels<B>::s;
+    constexpr float kMargin = 0x1p-14f;
+    const float tf = __fadd_rn(__fmul_rn(fabsf(g), k), u);
+    const float fl = floorf(tf);
+    const float d = __fsub_rn(tf, fl); // exact
+    // d in [2^-14, 1 - 2^-14], as one comparison (its rounding moves the
+    // bound by at most 2^-25, far inside the slack of the margin)
+    if (!(fabsf(__fsub_rn(d, 0.5f)) <= 0.5f - kMargin))
+        return qsgd_level_exact<B>(g, M, u);
+    return (int32_t)copysignf(fminf(fl, s), g); // g = -0 gives 0
 }
 
 // ------------------------------------------------------------------- max ----
@@ -143,6 +168,8 @@ __global__ void __launch_bounds__(kThreads)
 {
     using L = Levels<B>;
     const float M = *max_in;
+    const bool fast = M > 0.0f && M <= FLT_MAX;          // uniform over the grid
+    const float k = __fdiv_rn((float)L::s, M);
     if (blockIdx.x == 0 && threadIdx.x == 0) {
         compr[0] = bits_from_f32(M);
         compr[1] = bits_from_f32((float)B);
@@ -177,10 +204,18 @@ __global__ void __launch_bounds__(kThreads)
             const int64_t gi = g0 + j * kWarp + lane;
             const uint4 r = philox4x32_10(
                 make_uint4((uint32_t)gi, (uint32_t)((uint64_t)gi >> 32), 0u, 0u), key0, key1);
-            const uint32_t c0 = (uint32_t)qsgd_level<B>(gv[j].x, M, unit_draw(r.x)) & L::mask;
-            const uint32_t c1 = (uint32_t)qsgd_level<B>(gv[j].y, M, unit_draw(r.y)) & L::mask;
-            const uint32_t c2 = (uint32_t)qsgd_level<B>(gv[j].z, M, unit_draw(r.z)) & L::mask;
-            const uint32_t c3 = (uint32_t)qsgd_level<B>(gv[j].w, M, unit_draw(r.w)) & L::mask;
+            uint32_t c0, c1, c2, c3;
+            if (fast) {
+                c0 = (uint32_t)qsgd_level<B>(gv[j].x, M, k, unit_draw(r.x)) & L::mask;
+                c1 = (uint32_t)qsgd_level<B>(gv[j].y, M, k, unit_draw(r.y)) & L::mask;
+                c2 = (uint32_t)qsgd_level<B>(gv[j].z, M, k, unit_draw(r.z)) & L::mask;
+                c3 = (uint32_t)qsgd_level<B>(gv[j].w, M, k, unit_draw(r.w)) & L::mask;
+            } else {
+                c0 = (uint32_t)qsgd_level_exact<B>(gv[j].x, M, unit_draw(r.x)) & L::mask;
+                c1 = (uint32_t)qsgd_level_exact<B>(gv[j].y, M, unit_draw(r.y)) & L::mask;
+                c2 = (uint32_t)qsgd_level_exact<B>(gv[j].z, M, unit_draw(r.z)) & L::mask;
+                c3 = (uint32_t)qsgd_level_exact<B>(gv[j].w, M, unit_draw(r.w)) & L::mask;
+            }
             uint32_t piece = (c0 << (3 * B)) | (c1 << (2 * B)) | (c2 << B) | c3;
             // codes of elements >= n are zero
             const int64_t valid = n - 4 * gi;
@@ -200,66 +235,102 @@ __global__ void __launch_bounds__(kThreads)
 }
 
 // ----------------------------------------------------------------- merge ----
+// Integer sum of the W workers' levels, a whole record word at a time.  XOR
+// with the sign bit of every b-bit field turns a two's-complement level q
+// into q + 2^(b-1) in [0, 2^b); masking every fourth (b = 2, 4) or every
+// other (b = 8) field spreads the biased fields into 8-bit (b = 2) or 16-bit
+// lanes of 32-bit registers, where one integer add sums a lane group over a
+// worker without carries crossing lanes (at most 64 workers: 64 * 3 < 2^8,
+// 64 * 255 < 2^16).  At the end each lane's sum, minus W * 2^(b-1), is the
+// exact integer level sum, converted to binary32 exactly through the 2^23
+// magic number (it is below 2^23) and scaled once by fl(M / s).
+//
+// A thread owns whole words: word l of each 32-word block of its warp (for
+// b = 2, also word 32 + l, loaded together for more bytes in flight), and
+// stores its 32/b outputs as 128-bit (b = 8) or 256-bit rows.
+template <int B> struct Swar {
+    static constexpr int kFields = 32 / B;          // elements per word
+    static constexpr int kLaneBits = B == 2 ? 8 : 16;
+    static constexpr int kLanesPerReg = 32 / kLaneBits;
+    static constexpr int kRegs = kFields / kLanesPerReg;
+    static constexpr uint32_t kSign = B == 2 ? 0xAAAAAAAAu : (B == 4 ? 0x88888888u : 0x80808080u);
+    // fields j, j + kRegs, j + 2 kRegs, ... (counted from the least significant) -> register j
+    static constexpr uint32_t kMask = B == 2 ? 0x03030303u : (B == 4 ? 0x000F000Fu : 0x00FF00FFu);
+    static constexpr int kSlots = B == 2 ? 2 : 1;   // words per thread (measured best)
+};
+
 template <int B, bool kVec>
 __global__ void __launch_bounds__(kThreads)
     qsgd_merge_kernel(const __grid_constant__ RecordSet set, int W, float *__restrict__ out,
                       int64_t n)
 {
-    using L = Levels<B>;
+    using S = Swar<B>;
+    constexpr int kBatch = 8;
+    constexpr int kSlots = S::kSlots;
     __shared__ const uint32_t *s_payload[QGA_MAX_WORKERS];
     if (threadIdx.x < W)
         s_payload[threadIdx.x] = set.rec[threadIdx.x] + 3;
     __syncthreads();
-    const float step = __fdiv_rn(f32_from_bits(set.rec[0][0]), (float)L::s);
-    constexpr int LW = L::lanes_per_word;
+    const float step = __fdiv_rn(f32_from_bits(set.rec[0][0]), (float)Levels<B>::s);
+    // 2^23 + W 2^(b-1): the magic-number conversion's offset and the bias
+    const float offset = 8388608.0f + (float)(W << (B - 1));
+    const int64_t nwords = (n * B + 31) >> 5;
     const int lane = threadIdx.x & (kWarp - 1);
-    const int64_t groups = (n + 3) >> 2;
-    const int64_t tiles = (groups + kTileGroups - 1) / kTileGroups;
-    const int64_t stride = (int64_t)gridDim.x * kWarpsPerBlock;
-    for (int64_t tile = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5); tile < tiles;
-         tile += stride) {
-        const int64_t g0 = tile * kTileGroups;
-        int32_t acc[kGroupsPerLane][4] = {};
-        constexpr int kBatch = 8;
+    const int64_t nslices = (nwords + kWarp * kSlots - 1) / (kWarp * kSlots);
+    for (int64_t sl = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5; sl < nslices;
+         sl += ((int64_t)gridDim.x * kThreads) >> 5) {
+        uint32_t acc[kSlots][S::kRegs] = {};
+        int64_t kws[kSlots];
+#pragma unroll
+        for (int t = 0; t < kSlots; ++t)
+            kws[t] = sl * (kWarp * kSlots) + t * kWarp + lane;
         for (int wb = 0; wb < W; wb += kBatch) {
-            uint32_t words[kBatch][kGroupsPerLane];
+            uint32_t words[kSlots][kBatch];
 #pragma unroll
-            for (int k = 0; k < kBatch; ++k)
+            for (int i = 0; i < kBatch; ++i)
 #pragma unroll
-                for (int j = 0; j < kGroupsPerLane; ++j) {
-                    const int64_t gi = g0 + j * kWarp + lane;
-                    words[k][j] = (wb + k < W && gi < groups) ? ld_stream_u32(s_payload[wb + k] + gi / LW)
-                                                              : 0u;
-                }
+                for (int t = 0; t < kSlots; ++t)
+                    words[t][i] = (wb + i < W && kws[t] < nwords)
+                                      ? ld_stream_u32(s_payload[wb + i] + kws[t]) : 0u;
 #pragma unroll
-            for (int k = 0; k < kBatch; ++k) {
-                if (wb + k < W) { // warp-uniform
+            for (int i = 0; i < kBatch; ++i) {
+                if (wb + i >= W) // warp-uniform
+                    break;
 #pragma unroll
-                    for (int j = 0; j < kGroupsPerLane; ++j) {
-                        // this group's 4B bits, moved to the top of the word
-                        const uint32_t top = words[k][j] << (4 * B * (lane % LW));
+                for (int t = 0; t < kSlots; ++t) {
+                    const uint32_t biased = words[t][i] ^ S::kSign;
 #pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            acc[j][e] += (int32_t)(top << (B * e)) >> (32 - B);
-                    }
+                    for (int j = 0; j < S::kRegs; ++j)
+                        acc[t][j] += (biased >> (B * j)) & S::kMask;
                 }
             }
         }
 #pragma unroll
-        for (int j = 0; j < kGroupsPerLane; ++j) {
-            const int64_t gi = g0 + j * kWarp + lane;
-            const float4 v = make_float4(__fmul_rn(__int2float_rn(acc[j][0]), step),
-                                         __fmul_rn(__int2float_rn(acc[j][1]), step),
-                                         __fmul_rn(__int2float_rn(acc[j][2]), step),
-                                         __fmul_rn(__int2float_rn(acc[j][3]), step));
-            if (kVec && gi < (n >> 2)) {
-                st_stream_f4(out + 4 * gi, v);
-            } else {
-                const float vv[4] = {v.x, v.y, v.z, v.w};
+        for (int t = 0; t < kSlots; ++t) {
+            const int64_t kw = kws[t];
+            if (kw >= nwords)
+                continue;
+            float v[S::kFields];
 #pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    if (4 * gi + k < n)
-                        st_stream_f1(out + 4 * gi + k, vv[k]);
+            for (int e = 0; e < S::kFields; ++e) {
+                const int f = S::kFields - 1 - e; // element e sits in field f from the bottom
+                const uint32_t sum = (acc[t][f % S::kRegs] >> (S::kLaneBits * (f / S::kRegs))) &
+                                     ((1u << S::kLaneBits) - 1u);
+                v[e] = __fmul_rn(__fsub_rn(__uint_as_float(0x4B000000u | sum), offset), step);
+            }
+            const int64_t e0 = kw * S::kFields;
+            if (kVec && e0 + S::kFields <= n) {
+                if (S::kFields == 4)
+                    st_stream_f4(out + e0, make_float4(v[0], v[1], v[2], v[3]));
+                else
+#pragma unroll
+                    for (int c = 0; c < S::kFields; c += 8)
+                        st_stream_f8(out + e0 + c, v + c);
+            } else {
+#pragma unroll
+                for (int e = 0; e < S::kFields; ++e)
+                    if (e0 + e < n)
+                        st_stream_f1(out + e0 + e, v[e]);
             }
         }
     }
@@ -270,6 +341,14 @@ std::atomic<int> occ_q[3][2][64];
 std::atomic<int> occ_m[3][2][64];
 
 int bits_slot(int bits) { return bits == 2 ? 0 : (bits == 4 ? 1 : (bits == 8 ? 2 : -1)); }
+
+template <int B>
+unsigned merge_grid(int64_t n, int resident)
+{
+    const int64_t nwords = (n * B + 31) >> 5;
+    const int64_t per_block = (int64_t)kThreads * Swar<B>::kSlots;
+    return grid_for((nwords + per_block - 1) / per_block, resident);
+}
 
 unsigned group_grid(int64_t n, int resident)
 {
@@ -299,13 +378,13 @@ template <int B>
 void launch_merge(const RecordSet &set, int W, float *out, int64_t n, cudaStream_t stream)
 {
     const int s = bits_slot(B);
-    if (aligned(out, 16)) {
+    if (aligned(out, 32)) {
         auto k = qsgd_merge_kernel<B, true>;
-        k<<<group_grid(n, resident_blocks(k, kThreads, occ_m[s][0])), kThreads, 0, stream>>>(
+        k<<<merge_grid<B>(n, resident_blocks(k, kThreads, occ_m[s][0])), kThreads, 0, stream>>>(
             set, W, out, n);
     } else {
         auto k = qsgd_merge_kernel<B, false>;
-        k<<<group_grid(n, resident_blocks(k, kThreads, occ_m[s][1])), kThreads, 0, stream>>>(
+        k<<<merge_grid<B>(n, resident_blocks(k, kThreads, occ_m[s][1])), kThreads, 0, stream>>>(
             set, W, out, n);
     }
 }

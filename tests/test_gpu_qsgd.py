@@ -189,3 +189,30 @@ def test_qsgd_128M_eight_workers_sampled():
         np.testing.assert_allclose(got, want, rtol=AGG_RTOL, atol=AGG_ATOL)
         assert same_bits_f32(got, want)
         del comprs
+
+
+@pytest.mark.parametrize("b", BITS)
+def test_quantize_levels_next_to_integer_boundaries(b):
+    """Inputs placed so that |g|/M*s + u falls just above or below an integer
+    (within 1e-7 .. 2e-4 of it), where a shortcut in the level computation
+    would first disagree with the definition's three operations."""
+    q = qga()
+    s = 2 ** (b - 1) - 1
+    M = np.float32(3.0)
+    seed = 987654321
+    n = 4096
+    rng = np.random.default_rng(b)
+    deltas = np.array([1e-7, -1e-7, 3e-6, -3e-6, 2e-5, -2e-5, 4e-5, -4e-5, 6e-5, -6e-5, 1e-4, -2e-4])
+    g = np.empty(n, np.float32)
+    for e in range(n):
+        u = oracle.qsgd_uniform(seed, e)
+        target = rng.integers(0, s + 1) + deltas[e % deltas.size]
+        x = np.float32(max(0.0, (target - u)) * float(M) / s)
+        g[e] = -x if rng.random() < 0.5 else x
+    g[:2] = [float(M), -float(M)]
+    dev_g = torch.from_numpy(g).to(DEV)
+    Md = torch.tensor([float(M)], device=DEV)
+    c = torch.empty(q.qga_qsgd_words(n, b), dtype=torch.int32, device=DEV)
+    q.qga_qsgd_mn_quantize(dev_g, c, b, seed, Md)
+    want = oracle.qsgd_mn_quantize(g, b, seed, M)
+    assert np.array_equal(u32(c), want), first_diff(u32(c), want)
