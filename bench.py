@@ -42,10 +42,12 @@ WORKLOAD = "vgg16-8w"
 QUANT_BYTES_PER_ELEM = 12.25        # read g 4 + read r 4 + write r 4 + write codes 0.25
 FALLBACK_HBM_GBS = 6650.0
 
-# dram__bytes_read.sum + dram__bytes_write.sum per element of the quantize
-# kernel, from the ncu capture in profiles/, keyed by the hash of the CUDA
-# sources it was taken on (reported as null once the kernel has changed).
-MEASURED_TRAFFIC = {}
+# dram__bytes_read.sum + dram__bytes_write.sum per element of one full-size
+# launch of the quantize kernel (profiles/quantize_2bit_kernel_fp32_vgg16.md),
+# keyed by the hash of the sources that kernel is compiled from; reported as
+# null once they have changed since the capture.
+MEASURED_TRAFFIC = {"1b60ae20dff0ea9c": 11.905}   # 1.6469 GB per launch of n = 138,357,544
+QUANT_SOURCES = ("qga_common.cuh", "qga_2bit_tiles.cuh", "qga_2bit.cu")
 
 
 def parse_args():
@@ -64,10 +66,13 @@ def parse_args():
     return p.parse_args()
 
 
-def csrc_hash():
+def csrc_hash(names=None):
+    """Hash of the CUDA sources (all of them, or the named files)."""
     h = hashlib.sha256()
     pkg = os.path.join(ROOT, "quantized_gradient_aggregation_b200", "csrc")
-    for path in sorted(glob.glob(os.path.join(pkg, "*.cu*"))):
+    paths = sorted(glob.glob(os.path.join(pkg, "*.cu*"))) if names is None else \
+        [os.path.join(pkg, x) for x in names]
+    for path in paths:
         with open(path, "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -341,7 +346,7 @@ def run_qga(args, rank, world, local_rank):
     peak, peak_kind = measured_peaks()
     quant_gbs = QUANT_BYTES_PER_ELEM * n / (quant_ms * 1e-3) / 1e9
     merge_gbs = (0.25 * W + 4) * n / (merge_ms * 1e-3) / 1e9
-    traffic_per_elem = MEASURED_TRAFFIC.get(csrc_hash())
+    traffic_per_elem = MEASURED_TRAFFIC.get(csrc_hash(QUANT_SOURCES))
     line = {
         "metric": METRIC,
         "value": job_gelem_per_s(world, W, n, K, total_ms),
@@ -369,6 +374,7 @@ def run_qga(args, rank, world, local_rank):
         "gpu_launches": K * (W + 1),
         "clocks": clocks,
         "csrc": csrc_hash(),
+        "quantize_sources": csrc_hash(QUANT_SOURCES),
     }
     if rows is not None:
         line["kernels"].update(rows)

@@ -6,9 +6,10 @@
 // one after the other, so a bucket can be split back into per-tensor records
 // without copying.
 //
-// Work distribution.  Each tensor is cut into chunks of 8192 elements (16
-// warp tiles; a tensor of n = 0 still owns one chunk, which writes its
-// header).  The host numbers the chunks of all tensors consecutively and
+// Work distribution.  Each tensor is cut into chunks (8192 elements for the
+// quantizer, 32768 for the merge, whose blocks rebuild a per-worker table at
+// every chunk; a tensor of n = 0 still owns one quantizer chunk, which writes
+// its header).  The host numbers the chunks of all tensors consecutively and
 // passes the descriptor table BY VALUE as a kernel parameter (no device
 // table, no allocation, no copy): a persistent grid strides over the chunk
 // numbers, and each block finds its tensor by a binary search over the
@@ -22,7 +23,8 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarpsPerBlock = kThreads / kWarp;
-constexpr int64_t kChunkElems = 8192; // a whole number of quantize tiles and merge slices
+constexpr int64_t kChunkElems = 8192;       // quantize: a whole number of quantize tiles
+constexpr int64_t kMergeChunkElems = 32768; // merge: 4 slices per warp between block barriers
 constexpr int kMaxRows = 256;
 
 struct QuantRow {
@@ -115,7 +117,7 @@ __global__ void __launch_bounds__(kThreads, 3)
     __shared__ float s_neg[QGA_MAX_WORKERS], s_pos[QGA_MAX_WORKERS];
     __shared__ float2 s_table[QGA_MAX_WORKERS][16];
     __shared__ float4 s_stage[kWarpsPerBlock][kStagePerWarp];
-    constexpr int64_t kChunkSlices = kChunkElems / kSliceElems;
+    constexpr int64_t kChunkSlices = kMergeChunkElems / kSliceElems;
     const int lane = threadIdx.x & (kWarp - 1);
     const int warp = threadIdx.x >> 5;
     for (int64_t chunk = blockIdx.x; chunk < tab.total_chunks; chunk += gridDim.x) {
@@ -176,9 +178,9 @@ void launch_bucket_merge_any(const MergeTable &tab, float *out, cudaStream_t str
     }
 }
 
-int64_t chunks_of(int64_t n, bool at_least_one)
+int64_t chunks_of(int64_t n, bool at_least_one, int64_t chunk_elems = kChunkElems)
 {
-    const int64_t c = (n + kChunkElems - 1) / kChunkElems;
+    const int64_t c = (n + chunk_elems - 1) / chunk_elems;
     return (at_least_one && c == 0) ? 1 : c;
 }
 
@@ -302,7 +304,7 @@ extern "C" int qga_dequant_accumulate_2bit_bucket(const uint32_t *const *compr, 
             r.elem_off = elem_off;
             r.chunk_begin = chunk;
             r.vec = aligned(out + elem_off, 16);
-            chunk += chunks_of(r.n, false);
+            chunk += chunks_of(r.n, false, kMergeChunkElems);
             word_off += 3 + (r.n + 15) / 16;
             elem_off += r.n;
         }

@@ -259,6 +259,48 @@ template <int B> struct Swar {
     static constexpr int kSlots = B == 2 ? 2 : 1;   // words per thread (measured best)
 };
 
+// Outputs of one record word from its lane sums: element e sits in field
+// kFields - 1 - e (counted from the least significant).
+template <int B, bool kVec>
+__device__ __forceinline__ void merge_store_word(const uint32_t (&acc)[Swar<B>::kRegs], int64_t kw,
+                                                 float offset, float step, float *__restrict__ out,
+                                                 int64_t n)
+{
+    using S = Swar<B>;
+    float v[S::kFields];
+#pragma unroll
+    for (int e = 0; e < S::kFields; ++e) {
+        const int f = S::kFields - 1 - e;
+        const uint32_t sum =
+            (acc[f % S::kRegs] >> (S::kLaneBits * (f / S::kRegs))) & ((1u << S::kLaneBits) - 1u);
+        v[e] = __fmul_rn(__fsub_rn(__uint_as_float(0x4B000000u | sum), offset), step);
+    }
+    const int64_t e0 = kw * S::kFields;
+    if (kVec && e0 + S::kFields <= n) {
+        if (S::kFields == 4)
+            st_stream_f4(out + e0, make_float4(v[0], v[1], v[2], v[3]));
+        else
+#pragma unroll
+            for (int c = 0; c < S::kFields; c += 8)
+                st_stream_f8(out + e0 + c, v + c);
+    } else {
+#pragma unroll
+        for (int e = 0; e < S::kFields; ++e)
+            if (e0 + e < n)
+                st_stream_f1(out + e0 + e, v[e]);
+    }
+}
+
+template <int B>
+__device__ __forceinline__ void merge_add_word(uint32_t (&acc)[Swar<B>::kRegs], uint32_t word)
+{
+    using S = Swar<B>;
+    const uint32_t biased = word ^ S::kSign;
+#pragma unroll
+    for (int j = 0; j < S::kRegs; ++j)
+        acc[j] += (biased >> (B * j)) & S::kMask;
+}
+
 template <int B, bool kVec>
 __global__ void __launch_bounds__(kThreads)
     qsgd_merge_kernel(const __grid_constant__ RecordSet set, int W, float *__restrict__ out,
@@ -266,7 +308,6 @@ __global__ void __launch_bounds__(kThreads)
 {
     using S = Swar<B>;
     constexpr int kBatch = 8;
-    constexpr int kSlots = S::kSlots;
     __shared__ const uint32_t *s_payload[QGA_MAX_WORKERS];
     if (threadIdx.x < W)
         s_payload[threadIdx.x] = set.rec[threadIdx.x] + 3;
@@ -275,63 +316,52 @@ __global__ void __launch_bounds__(kThreads)
     // 2^23 + W 2^(b-1): the magic-number conversion's offset and the bias
     const float offset = 8388608.0f + (float)(W << (B - 1));
     const int64_t nwords = (n * B + 31) >> 5;
-    const int lane = threadIdx.x & (kWarp - 1);
-    const int64_t nslices = (nwords + kWarp * kSlots - 1) / (kWarp * kSlots);
-    for (int64_t sl = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5; sl < nslices;
-         sl += ((int64_t)gridDim.x * kThreads) >> 5) {
-        uint32_t acc[kSlots][S::kRegs] = {};
-        int64_t kws[kSlots];
+    const int64_t stride = (int64_t)gridDim.x * kThreads;
+    if constexpr (S::kSlots == 1) {
+        for (int64_t kw = (int64_t)blockIdx.x * kThreads + threadIdx.x; kw < nwords; kw += stride) {
+            uint32_t acc[S::kRegs] = {};
+            for (int wb = 0; wb < W; wb += kBatch) {
+                uint32_t words[kBatch];
 #pragma unroll
-        for (int t = 0; t < kSlots; ++t)
-            kws[t] = sl * (kWarp * kSlots) + t * kWarp + lane;
-        for (int wb = 0; wb < W; wb += kBatch) {
-            uint32_t words[kSlots][kBatch];
+                for (int i = 0; i < kBatch; ++i)
+                    words[i] = wb + i < W ? ld_stream_u32(s_payload[wb + i] + kw) : 0u;
 #pragma unroll
-            for (int i = 0; i < kBatch; ++i)
-#pragma unroll
-                for (int t = 0; t < kSlots; ++t)
-                    words[t][i] = (wb + i < W && kws[t] < nwords)
-                                      ? ld_stream_u32(s_payload[wb + i] + kws[t]) : 0u;
-#pragma unroll
-            for (int i = 0; i < kBatch; ++i) {
-                if (wb + i >= W) // warp-uniform
-                    break;
-#pragma unroll
-                for (int t = 0; t < kSlots; ++t) {
-                    const uint32_t biased = words[t][i] ^ S::kSign;
-#pragma unroll
-                    for (int j = 0; j < S::kRegs; ++j)
-                        acc[t][j] += (biased >> (B * j)) & S::kMask;
+                for (int i = 0; i < kBatch; ++i) {
+                    if (wb + i >= W) // warp-uniform
+                        break;
+                    merge_add_word<B>(acc, words[i]);
                 }
             }
+            merge_store_word<B, kVec>(acc, kw, offset, step, out, n);
         }
+    } else {
+        // a warp takes 2 x 32 consecutive words: lane l the words l and 32 + l,
+        // loaded together for more bytes in flight
+        const int lane = threadIdx.x & (kWarp - 1);
+        const int64_t nslices = (nwords + 2 * kWarp - 1) / (2 * kWarp);
+        for (int64_t sl = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5; sl < nslices;
+             sl += stride >> 5) {
+            const int64_t k0 = sl * (2 * kWarp) + lane, k1 = k0 + kWarp;
+            uint32_t acc0[S::kRegs] = {}, acc1[S::kRegs] = {};
+            for (int wb = 0; wb < W; wb += kBatch) {
+                uint32_t w0[kBatch], w1[kBatch];
 #pragma unroll
-        for (int t = 0; t < kSlots; ++t) {
-            const int64_t kw = kws[t];
-            if (kw >= nwords)
-                continue;
-            float v[S::kFields];
+                for (int i = 0; i < kBatch; ++i) {
+                    w0[i] = (wb + i < W && k0 < nwords) ? ld_stream_u32(s_payload[wb + i] + k0) : 0u;
+                    w1[i] = (wb + i < W && k1 < nwords) ? ld_stream_u32(s_payload[wb + i] + k1) : 0u;
+                }
 #pragma unroll
-            for (int e = 0; e < S::kFields; ++e) {
-                const int f = S::kFields - 1 - e; // element e sits in field f from the bottom
-                const uint32_t sum = (acc[t][f % S::kRegs] >> (S::kLaneBits * (f / S::kRegs))) &
-                                     ((1u << S::kLaneBits) - 1u);
-                v[e] = __fmul_rn(__fsub_rn(__uint_as_float(0x4B000000u | sum), offset), step);
+                for (int i = 0; i < kBatch; ++i) {
+                    if (wb + i >= W) // warp-uniform
+                        break;
+                    merge_add_word<B>(acc0, w0[i]);
+                    merge_add_word<B>(acc1, w1[i]);
+                }
             }
-            const int64_t e0 = kw * S::kFields;
-            if (kVec && e0 + S::kFields <= n) {
-                if (S::kFields == 4)
-                    st_stream_f4(out + e0, make_float4(v[0], v[1], v[2], v[3]));
-                else
-#pragma unroll
-                    for (int c = 0; c < S::kFields; c += 8)
-                        st_stream_f8(out + e0 + c, v + c);
-            } else {
-#pragma unroll
-                for (int e = 0; e < S::kFields; ++e)
-                    if (e0 + e < n)
-                        st_stream_f1(out + e0 + e, v[e]);
-            }
+            if (k0 < nwords)
+                merge_store_word<B, kVec>(acc0, k0, offset, step, out, n);
+            if (k1 < nwords)
+                merge_store_word<B, kVec>(acc1, k1, offset, step, out, n);
         }
     }
 }

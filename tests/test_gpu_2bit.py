@@ -253,3 +253,29 @@ def test_vgg16_eight_workers_five_iterations_sampled():
             np.testing.assert_allclose(got, want, rtol=AGG_RTOL, atol=AGG_ATOL)
             assert same_bits_f32(got, want), (it, int(pick[i]))
             at += m
+
+
+def test_residual_checkpoint_resume():
+    """The only state of the method is the caller's residual: saving it to
+    the host mid-run and restoring it into a fresh buffer continues the run
+    word for word."""
+    q = qga()
+    w = workloads.WORKLOADS["ef2bit-1M"]
+    n = 100_003
+    grads = workloads.gradient_stream(w, 6, device=DEV, n=n)
+    words = q.qga_2bit_words(n)
+    r = torch.zeros(n, device=DEV)
+    c = torch.empty(words, dtype=torch.int32, device=DEV)
+    for it in range(3):
+        q.qga_quantize_2bit(grads[it], r, c, w.neg_thr, w.pos_thr)
+    saved = r.cpu().clone()
+    straight = []
+    for it in range(3, 6):
+        q.qga_quantize_2bit(grads[it], r, c, w.neg_thr, w.pos_thr)
+        straight.append(u32(c).copy())
+    r2 = saved.to(DEV)
+    c2 = torch.empty(words, dtype=torch.int32, device=DEV)
+    for k, it in enumerate(range(3, 6)):
+        q.qga_quantize_2bit(grads[it], r2, c2, w.neg_thr, w.pos_thr)
+        assert np.array_equal(u32(c2), straight[k]), it
+    assert same_bits_f32(f32(r2), f32(r))
