@@ -88,6 +88,11 @@ def _declare(L):
     L.oracle_qsgd_words.argtypes = [i64, i32]
     L.oracle_qsgd_mn_quantize.argtypes = [vp, vp, i64, i32, u64, f32]
     L.oracle_qsgd_mn_dequant_accumulate.argtypes = [vp, i32, vp, i64, i32]
+    L.oracle_ternary_words.restype = i64
+    L.oracle_ternary_words.argtypes = [i64]
+    L.oracle_quantize_ternary.argtypes = [vp, vp, vp, i64, f32, f32]
+    L.oracle_dequantize_ternary.argtypes = [vp, vp, i64]
+    L.oracle_dequant_accumulate_ternary.argtypes = [vp, i32, vp, i64]
     return L
 
 
@@ -221,4 +226,38 @@ def qsgd_mn_dequant_accumulate(comprs, n, b, L=None):
     comprs = [_c(c, np.uint32) for c in comprs]
     out = np.empty(n, np.float32)
     L.oracle_qsgd_mn_dequant_accumulate(_ptr_array(comprs), len(comprs), out.ctypes.data, n, b)
+    return out
+
+
+# -------------------------------------------------------- dense ternary ----
+
+def words_ternary(n: int) -> int:
+    return int(lib().oracle_ternary_words(n))
+
+
+def quantize_ternary(grad, residual, neg_thr, pos_thr, L=None):
+    """Return (compr, new_residual) of the dense ternary record."""
+    L = L or lib()
+    grad = _c(grad, np.float32)
+    res = _c(residual, np.float32).copy()
+    n = res.size
+    compr = np.zeros(int(L.oracle_ternary_words(n)), np.uint32)
+    L.oracle_quantize_ternary(grad.ctypes.data, res.ctypes.data, compr.ctypes.data, n,
+                              float(neg_thr), float(pos_thr))
+    return compr, res
+
+
+def dequantize_ternary(compr, n, L=None):
+    L = L or lib()
+    compr = _c(compr, np.uint32)
+    out = np.empty(n, np.float32)
+    L.oracle_dequantize_ternary(compr.ctypes.data, out.ctypes.data, n)
+    return out
+
+
+def dequant_accumulate_ternary(comprs, n, L=None):
+    L = L or lib()
+    comprs = [_c(c, np.uint32) for c in comprs]
+    out = np.empty(n, np.float32)
+    L.oracle_dequant_accumulate_ternary(_ptr_array(comprs), len(comprs), out.ctypes.data, n)
     return out

@@ -372,3 +372,71 @@ void oracle_qsgd_mn_dequant_accumulate(const uint32_t *const *compr, int W, floa
         out[e] = (float)sum * step;
     }
 }
+
+/* ------------------------------------------------------------------ */
+/* Dense ternary packing of the 2-bit threshold codes                  */
+/* ------------------------------------------------------------------ */
+/* [MX] "Two bit quantization" notes that three values need only log2(3)
+ * bits and leaves the wasted code for later.  This library's dense format:
+ * the three codes 00, 01, 10 become the trits 0, 1, 2; five consecutive
+ * elements form one byte as the base-3 numeral t0 t1 t2 t3 t4 (element 0 the
+ * most significant trit, so a byte is at most 242); payload byte j holds
+ * elements 5j..5j+4 and sits at byte 12 + j of the record (memory order)
+ * after the same three-word header [neg, pos, n]; the record is padded to
+ * whole 32-bit words, and trits past n and padding bytes are zero.  The
+ * error feedback is exactly that of the 2-bit operator. */
+
+int64_t oracle_ternary_words(int64_t n)
+{
+    return 3 + (n + 19) / 20;
+}
+
+void oracle_quantize_ternary(const float *grad, float *residual, uint32_t *compr, int64_t n,
+                             float neg_thr, float pos_thr)
+{
+    unsigned char *payload = (unsigned char *)(compr + 3);
+    write_2bit_header(compr, n, neg_thr, pos_thr);
+    for (int64_t w = 0; w < (n + 19) / 20; ++w)
+        compr[3 + w] = 0u;
+    for (int64_t j = 0; 5 * j < n; ++j) {
+        unsigned value = 0;
+        for (int64_t e = 5 * j; e < 5 * j + 5; ++e) {
+            unsigned trit = 0;
+            if (e < n)
+                trit = quantize_one(grad[e], &residual[e], neg_thr, pos_thr);
+            value = value * 3 + trit;
+        }
+        payload[j] = (unsigned char)value;
+    }
+}
+
+/* Trit of element e: digit e mod 5 (most significant first) of byte e / 5. */
+static uint32_t ternary_code_at(const uint32_t *compr, int64_t e)
+{
+    const unsigned char *payload = (const unsigned char *)(compr + 3);
+    unsigned value = payload[e / 5];
+    for (int64_t k = e % 5; k < 4; ++k)
+        value /= 3;
+    return value % 3;
+}
+
+void oracle_dequantize_ternary(const uint32_t *compr, float *out, int64_t n)
+{
+    float neg_thr = float_of(compr[0]);
+    float pos_thr = float_of(compr[1]);
+    for (int64_t e = 0; e < n; ++e)
+        out[e] = two_bit_value(ternary_code_at(compr, e), neg_thr, pos_thr);
+}
+
+void oracle_dequant_accumulate_ternary(const uint32_t *const *compr, int W, float *out, int64_t n)
+{
+    for (int64_t e = 0; e < n; ++e) {
+        float sum = 0.0f;
+        for (int w = 0; w < W; ++w) {
+            float neg_thr = float_of(compr[w][0]);
+            float pos_thr = float_of(compr[w][1]);
+            sum = sum + two_bit_value(ternary_code_at(compr[w], e), neg_thr, pos_thr);
+        }
+        out[e] = sum;
+    }
+}

@@ -488,4 +488,94 @@ def pin_qsgd_merge_identity(L):
             assert out[e] == want, (b, e, out[e], want)
 
 
+# ======================================================= dense ternary ====
+
+def _ternary_bytes(compr, nbytes):
+    return [int(b) for b in compr[3:].view(np.uint8)[:nbytes]]
+
+
+def _base3_digits(byte):
+    digits = []
+    for _ in range(5):
+        byte, d = divmod(byte, 3)
+        digits.append(d)
+    return digits[::-1]
+
+
+def pin_ternary_matches_2bit(L):
+    """The dense record carries exactly the 2-bit operator's codes (a pinned
+    routine) and leaves exactly its residual."""
+    rng = np.random.default_rng(37)
+    for n in (0, 1, 4, 5, 6, 19, 20, 21, 99, 1000):
+        g = (rng.standard_normal(n) * 0.6).astype(np.float32)
+        r = rng.uniform(-0.5, 0.5, n).astype(np.float32)
+        c2, r2 = oracle.quantize_2bit(g, r, -0.5, 0.5, L)
+        c3, r3 = oracle.quantize_ternary(g, r, -0.5, 0.5, L)
+        assert np.array_equal(r2.view(np.uint32), r3.view(np.uint32)), n
+        assert c3.size == 3 + -(-n // 20) == int(L.oracle_ternary_words(n))
+        assert c3[:3].tolist() == c2[:3].tolist()
+        trits = [d for b in _ternary_bytes(c3, -(-n // 5)) for d in _base3_digits(b)]
+        codes = [(int(c2[3 + e // 16]) >> (30 - 2 * (e % 16))) & 3 for e in range(n)]
+        assert trits[:n] == codes, n
+        assert not any(trits[n:])
+        # padding bytes past the last element's byte are zero
+        assert not any(int(b) for b in c3[3:].view(np.uint8)[-(-n // 5):])
+
+
+def pin_ternary_numeral(L):
+    """All 3^5 trit patterns: a byte is the base-3 numeral of its five codes,
+    first element most significant; the worked example's codes give bytes
+    34 and 18 (word 0x00001222)."""
+    gold = read_golden("two_bit_worked_example.txt")
+    codes = [int(c, 2) for c in gold["codes"].split()]
+    g = np.array([1.0, 2.5, -1.0, -3.0, 2.0, 0.5, 0.0, -2.0], np.float32)
+    c, _ = oracle.quantize_ternary(g, np.zeros(8, np.float32), -2.0, 2.0, L)
+    want = [0, 0]
+    for i, t in enumerate(codes + [0, 0]):
+        want[i // 5] = want[i // 5] * 3 + t
+    assert _ternary_bytes(c, 2) == want == [34, 18]
+    assert int(c[3]) == 0x1222
+    patterns = np.array(np.meshgrid(*[[0, 1, 2]] * 5, indexing="ij")).reshape(5, -1).T
+    codes = patterns.reshape(-1)                     # 243 * 5 elements
+    vals = np.where(codes == 1, 1.5, np.where(codes == 2, -0.75, 0.0)).astype(np.float32)
+    c, r = oracle.quantize_ternary(vals, np.zeros(vals.size, np.float32), -0.75, 1.5, L)
+    assert not r.any()
+    assert _ternary_bytes(c, 243) == list(range(243))
+    assert np.array_equal(oracle.dequantize_ternary(c, vals.size, L), vals)
+
+
+def pin_ternary_dequantize_and_merge(L):
+    """Random bytes decode digit by digit; the merge of power-of-two
+    thresholds is the exact sum; W = 1 equals dequantize."""
+    rng = np.random.default_rng(41)
+    n = 5 * 61 + 3
+    pow2 = [0.25, 0.5, 1.0, 2.0]
+    recs, thr = [], []
+    for w in range(5):
+        a, b = -float(rng.choice(pow2)), float(rng.choice(pow2))
+        words = np.zeros(3 + -(-n // 20), np.uint32)
+        words[:3] = np.array([a, b, n], np.float32).view(np.uint32)
+        nbytes = -(-n // 5)
+        bytes_ = rng.integers(0, 243, nbytes).astype(np.uint8)
+        # trits past n stay zero
+        last = _base3_digits(int(bytes_[-1]))
+        keep = n - 5 * (nbytes - 1)
+        v = 0
+        for i, d in enumerate(last):
+            v = v * 3 + (d if i < keep else 0)
+        bytes_[-1] = v
+        words[3:].view(np.uint8)[:nbytes] = bytes_
+        recs.append(words)
+        thr.append((a, b))
+    out = oracle.dequantize_ternary(recs[0], n, L)
+    trits = [d for b in _ternary_bytes(recs[0], -(-n // 5)) for d in _base3_digits(b)]
+    assert out.tolist() == [code_value(t, *thr[0]) for t in trits[:n]]
+    assert np.array_equal(oracle.dequant_accumulate_ternary(recs[:1], n, L), out)
+    merged = oracle.dequant_accumulate_ternary(recs, n, L)
+    all_trits = [[d for b in _ternary_bytes(r, -(-n // 5)) for d in _base3_digits(b)] for r in recs]
+    for e in range(n):
+        total = sum(Fraction(code_value(all_trits[w][e], *thr[w])) for w in range(len(recs)))
+        assert Fraction(float(merged[e])) == total, e
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -37,10 +37,16 @@ MUTANTS = [
     ("decode values swapped", "    if (code == 1u)\n        return pos_thr;",
      "    if (code == 1u)\n        return neg_thr;"),
     ("merge in reverse worker order",
-     "for (int w = 0; w < W; ++w) {\n            float neg_thr = float_of(compr[w][0]);",
-     "for (int w = W - 1; w >= 0; --w) {\n            float neg_thr = float_of(compr[w][0]);"),
-    ("merge uses worker 0 thresholds", "            float pos_thr = float_of(compr[w][1]);",
-     "            float pos_thr = float_of(compr[0][1]);"),
+     "for (int w = 0; w < W; ++w) {\n            float neg_thr = float_of(compr[w][0]);\n"
+     "            float pos_thr = float_of(compr[w][1]);\n            sum = sum + two_bit_value(two_bit_code_at",
+     "for (int w = W - 1; w >= 0; --w) {\n            float neg_thr = float_of(compr[w][0]);\n"
+     "            float pos_thr = float_of(compr[w][1]);\n            sum = sum + two_bit_value(two_bit_code_at"),
+    ("merge uses worker 0 thresholds",
+     "            float pos_thr = float_of(compr[w][1]);\n            sum = sum + two_bit_value(two_bit_code_at",
+     "            float pos_thr = float_of(compr[0][1]);\n            sum = sum + two_bit_value(two_bit_code_at"),
+    ("ternary merge uses worker 0 thresholds",
+     "            float pos_thr = float_of(compr[w][1]);\n            sum = sum + two_bit_value(ternary_code_at",
+     "            float pos_thr = float_of(compr[0][1]);\n            sum = sum + two_bit_value(ternary_code_at"),
     ("bf16 widening shift", "return float_of((uint32_t)h << 16);",
      "return float_of((uint32_t)h << 15);"),
     ("bucket offset without header", "        offset += oracle_2bit_words(n[t]);",
@@ -64,6 +70,10 @@ MUTANTS = [
     ("no sign extension", "        q -= (int32_t)(1u << b);", "        q += 0;"),
     ("merge step 2^(b-1)", "float step = M / (float)qsgd_levels(b);",
      "float step = M / (float)(1 << (b - 1));"),
+    ("ternary base 4", "            value = value * 3 + trit;", "            value = value * 4 + trit;"),
+    ("ternary least significant first", "    for (int64_t k = e % 5; k < 4; ++k)\n        value /= 3;",
+     "    for (int64_t k = 0; k < e % 5; ++k)\n        value /= 3;"),
+    ("ternary words per 16", "    return 3 + (n + 19) / 20;", "    return 3 + (n + 15) / 16;"),
 ]
 
 
