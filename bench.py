@@ -438,7 +438,23 @@ def time_rows(dev, stream, peak, reps=20):
     t = _time_launches(stream, lambda: ok(L.qga_dequantize_2bit(vp(c.data_ptr()), vp(out.data_ptr()),
                                                                 n, sp), "dequantize"), reps)
     rows["dequantize_2bit"] = _row(t, n, 4.25, peak, reps + 3, workload="vgg16 record, n=138,357,544")
-    del g, r, c, out
+    del c
+
+    # dense ternary records (5 codes per byte): quantize and the 8-worker merge
+    ct = [torch.empty(q.qga_ternary_words(n), dtype=torch.int32, device=dev) for _ in range(w.workers)]
+    t = _time_launches(stream, lambda: ok(L.qga_quantize_ternary(
+        vp(g.data_ptr()), vp(r.data_ptr()), vp(ct[0].data_ptr()), n, w.neg_thr, w.pos_thr, sp),
+        "quantize_ternary"), reps)
+    rows["quantize_ternary"] = _row(t, n, 12.2, peak, reps + 3, workload="vgg16 gradient, n=138,357,544")
+    for k in range(1, w.workers):
+        ct[k].copy_(ct[0])
+    tarr = (ctypes.c_void_p * w.workers)(*[cc.data_ptr() for cc in ct])
+    tp = ctypes.cast(tarr, ctypes.POINTER(ctypes.c_void_p))
+    t = _time_launches(stream, lambda: ok(L.qga_dequant_accumulate_ternary(
+        tp, w.workers, vp(out.data_ptr()), n, sp), "merge_ternary"), reps)
+    rows["dequant_accumulate_ternary_w8"] = _row(t, n, 0.2 * w.workers + 4, peak, reps + 3,
+                                                 workload="8 dense records of n=138,357,544")
+    del g, r, out, ct
 
     # BERT-Base bucket: quantize (bf16 grad) and 4-worker merge
     wb = workloads.WORKLOADS["bert-bucket-4w"]

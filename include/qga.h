@@ -152,6 +152,32 @@ int qga_dequant_accumulate_2bit_bucket(const uint32_t *const *compr, int num_wor
                                        const int64_t *n, int num_tensors, float *out,
                                        cudaStream_t stream);
 
+/* ===================================================== dense ternary 2-bit ==
+ * [MX] "Two bit quantization" observes that three code values waste a bit
+ * and defers the fix.  Dense record (this library's format): the same codes
+ * 00 / 01 / 10 as trits 0 / 1 / 2, five elements per byte as the base-3
+ * numeral t0 t1 t2 t3 t4 (element 0 most significant; a byte is <= 242),
+ * payload byte j = elements 5j..5j+4 at byte 12 + j of the record, after the
+ * same header [neg, pos, (float)n]; padded to whole words with zero bytes,
+ * trits past n zero.  0.2 bytes per element instead of 0.25.
+ *
+ * Words of a dense record: 3 + ceil(n / 20).  QGA_ERR_INVALID_ARG for n < 0. */
+int64_t qga_ternary_words(int64_t n);
+
+/* qga_quantize_2bit's error feedback (same codes, same residual, bit for bit)
+ * written as a dense record.
+ *   grad float[n], residual float[n] (in place), compr uint32[qga_ternary_words(n)] */
+int qga_quantize_ternary(const float *grad, float *residual, uint32_t *compr, int64_t n,
+                         float neg_threshold, float pos_threshold, cudaStream_t stream);
+
+/* Dense-record dequantize: out[e] = value of element e's code. */
+int qga_dequantize_ternary(const uint32_t *compr, float *out, int64_t n, cudaStream_t stream);
+
+/* Dense-record merge: out[e] = sum over w of the values, from +0 in worker
+ * order 0..W-1 (the same sums as qga_dequant_accumulate_2bit). */
+int qga_dequant_accumulate_ternary(const uint32_t *const *compr, int num_workers, float *out,
+                                   int64_t n, cudaStream_t stream);
+
 /* ==================================================== QSGD-MaxNorm, b bits ==
  * QSGDMaxNorm is named in [GC]; this library defines it as follows.
  *   s = 2^(b-1) - 1,  M = max over all workers and elements of |g|.

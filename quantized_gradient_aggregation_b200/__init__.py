@@ -6,8 +6,8 @@ tensors have the dtype / device / size the entry point expects, passes their
 data pointers and the current CUDA stream, and raises ``QGAError`` on a
 non-zero status.  All computation happens in the library's CUDA kernels;
 there is no CPU path.  Importing this package without a built ``libqga.so``
-raises ImportError (build it with ``python -m
-quantized_gradient_aggregation_b200.build``).
+raises ImportError (build it with ``python
+quantized_gradient_aggregation_b200/build.py``).
 
 Methods: MXNet pull request #8342 "[WIP] 2bit gradient compression" (the 2-bit
 threshold quantizer with residual, its record format and the receiver-side
@@ -35,7 +35,7 @@ QGA_DTYPE_BF16 = 1
 if not os.path.exists(LIB_PATH):
     raise ImportError(
         f"libqga.so not found at {LIB_PATH}; build it with "
-        "`python -m quantized_gradient_aggregation_b200.build` (nvcc, sm_100a)")
+        "`python quantized_gradient_aggregation_b200/build.py` (nvcc, sm_100a)")
 
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -61,6 +61,10 @@ _SIGS = {
     "qga_quantize_2bit_bucket": (_i32, [ctypes.POINTER(qga_bucket_tensor), _i32, _i32, _vp, _vp]),
     "qga_dequant_accumulate_2bit_bucket": (_i32, [_VPP, _i32, ctypes.POINTER(ctypes.c_int64), _i32,
                                                   _vp, _vp]),
+    "qga_ternary_words": (_i64, [_i64]),
+    "qga_quantize_ternary": (_i32, [_vp, _vp, _vp, _i64, _f32, _f32, _vp]),
+    "qga_dequantize_ternary": (_i32, [_vp, _vp, _i64, _vp]),
+    "qga_dequant_accumulate_ternary": (_i32, [_VPP, _i32, _vp, _i64, _vp]),
     "qga_qsgd_words": (_i64, [_i64, _i32]),
     "qga_qsgd_mn_max": (_i32, [_VPP, _i32, _i64, _vp, _vp]),
     "qga_qsgd_mn_quantize": (_i32, [_vp, _vp, _i64, _i32, _u64, _vp, _vp]),
@@ -223,6 +227,46 @@ def qga_dequant_accumulate_2bit_bucket(comprs, sizes, out, stream=None):
     _check(_lib.qga_dequant_accumulate_2bit_bucket(arr, len(comprs), n, len(sizes), _ptr(out),
                                                    _stream(stream, out.device)),
            "qga_dequant_accumulate_2bit_bucket")
+
+
+# ======================================================= dense ternary ====
+
+def qga_ternary_words(n: int) -> int:
+    w = _lib.qga_ternary_words(n)
+    if w < 0:
+        raise QGAError(int(w), "qga_ternary_words")
+    return int(w)
+
+
+def qga_quantize_ternary(grad, residual, compr, neg_threshold, pos_threshold, stream=None):
+    """The 2-bit error-feedback step written as a dense (5 codes per byte) record."""
+    n = residual.numel()
+    _need(residual, torch.float32, None, "residual")
+    _need(grad, torch.float32, n, "grad")
+    _need(compr, torch.int32, qga_ternary_words(n), "compr")
+    _check(_lib.qga_quantize_ternary(_ptr(grad), _ptr(residual), _ptr(compr), n,
+                                     float(neg_threshold), float(pos_threshold),
+                                     _stream(stream, residual.device)), "qga_quantize_ternary")
+
+
+def qga_dequantize_ternary(compr, out, stream=None):
+    n = out.numel()
+    _need(out, torch.float32, None, "out")
+    _need(compr, torch.int32, qga_ternary_words(n), "compr")
+    _check(_lib.qga_dequantize_ternary(_ptr(compr), _ptr(out), n, _stream(stream, out.device)),
+           "qga_dequantize_ternary")
+
+
+def qga_dequant_accumulate_ternary(comprs, out, stream=None):
+    n = out.numel()
+    _need(out, torch.float32, None, "out")
+    words = qga_ternary_words(n)
+    for i, c in enumerate(comprs):
+        _need(c, torch.int32, words, f"compr[{i}]")
+    arr, keep = _ptr_array(comprs)
+    _check(_lib.qga_dequant_accumulate_ternary(arr, len(comprs), _ptr(out), n,
+                                               _stream(stream, out.device)),
+           "qga_dequant_accumulate_ternary")
 
 
 # ================================================================ QSGD ====

@@ -1,6 +1,8 @@
 """Build libqga.so (sm_100a) in-tree with nvcc.
 
-    python -m quantized_gradient_aggregation_b200.build [--force] [--verbose]
+    python quantized_gradient_aggregation_b200/build.py [--force] [--verbose]
+
+(Run it by path: importing the package loads the library this script builds.)
 
 The library is plain CUDA C++ behind the C ABI of include/qga.h; no torch
 headers are involved.  ``-fmad=false`` keeps every floating-point expression

@@ -1,0 +1,332 @@
+// qga_ternary.cu -- dense ternary records of the 2-bit threshold codes:
+// quantize (fp32 gradient), dequantize and the W-worker merge.
+//
+// MXNet pull request #8342 "[WIP] 2bit gradient compression", "Two bit
+// quantization", notes that the three code values need fewer than two bits
+// and leaves the wasted code for later.  This library's dense record keeps
+// the same codes (00, 01, 10 -> trits 0, 1, 2) and the same error feedback,
+// and packs five elements per byte as the base-3 numeral t0 t1 t2 t3 t4
+// (element 0 most significant): payload byte j holds elements 5j..5j+4 and
+// sits at byte 12 + j of the record, after the header [neg, pos, n]; four
+// bytes (20 elements) fill one 32-bit word, and unused trits and padding
+// bytes are zero.  Record: 3 + ceil(n / 20) words (0.2 bytes per element
+// instead of 0.25).
+//
+// Quantize geometry: a warp owns a tile of 640 elements (160 groups of 4,
+// five per lane, every load a coalesced 512-byte row) = 32 payload words.
+// Each lane writes its groups' codes as bytes to a per-warp shared buffer;
+// lane l then reads the 20 codes of word l (five conflict-free 32-bit
+// loads: the stride of 5 words is odd) and forms each payload byte with one
+// byte-wise dot product against the weights 81, 27, 9, 3 (plus the fifth
+// code).  Decode geometry: a lane owns one payload word (20 elements); a
+// 243-entry shared table turns each byte into the bit masks of its codes
+// 01 and 10, and the outputs leave through a shared stage (again stride 5,
+// conflict-free) as coalesced 128-bit rows.
+
+#include "qga_2bit_tiles.cuh"
+
+namespace qga {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarpsPerBlock = kThreads / kWarp;
+constexpr int kTGroups = 5;                             // groups of 4 per lane per tile
+constexpr int kTTileElems = kWarp * kTGroups * 4;        // 640 elements = 32 words
+constexpr uint32_t kWeights = 0x03091B51u;               // bytes 81, 27, 9, 3 (little endian)
+
+__device__ __forceinline__ int64_t warp_id() { return (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5); }
+__device__ __forceinline__ int64_t warp_stride() { return (int64_t)gridDim.x * kWarpsPerBlock; }
+
+// Payload word from 20 codes held one per byte in five 32-bit words (code of
+// element 4i + k in byte k of c[i]).
+__device__ __forceinline__ uint32_t pack_ternary_word(const uint32_t (&c)[5])
+{
+    uint32_t word = 0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        // codes 5k .. 5k+3 start at byte 5k: word 5k / 4, byte offset (5k) % 4 = k
+        const int i = (5 * k) >> 2, o = k;
+        const uint32_t four = o == 0 ? c[i] : __funnelshift_r(c[i], c[i + 1], 8 * o);
+        const uint32_t fifth = (c[(5 * k + 4) >> 2] >> (8 * ((5 * k + 4) & 3))) & 0xFFu;
+        word |= (uint32_t)__dp4a(four, kWeights, fifth) << (8 * k);
+    }
+    return word;
+}
+
+template <bool kVec>
+__global__ void __launch_bounds__(kThreads)
+    quantize_ternary_kernel(const float *__restrict__ grad, float *__restrict__ residual,
+                            uint32_t *__restrict__ compr, int64_t n, float neg, float pos)
+{
+    __shared__ uint32_t s_codes[kWarpsPerBlock][kTTileElems / 4];
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        compr[0] = bits_from_f32(neg);
+        compr[1] = bits_from_f32(pos);
+        compr[2] = bits_from_f32(__ll2float_rn(n));
+    }
+    uint32_t *payload = compr + 3;
+    uint32_t *codes = s_codes[threadIdx.x >> 5];
+    const int lane = threadIdx.x & (kWarp - 1);
+    const int64_t full_groups = n >> 2;
+    const int64_t nwords = (n + 19) / 20;
+    const int64_t tiles = (n + kTTileElems - 1) / kTTileElems;
+    for (int64_t t = warp_id(); t < tiles; t += warp_stride()) {
+        const int64_t g0 = t * (kWarp * kTGroups);
+        float4 gv[kTGroups], rv[kTGroups];
+#pragma unroll
+        for (int j = 0; j < kTGroups; ++j) {
+            const int64_t gi = g0 + j * kWarp + lane;
+            if (kVec && gi < full_groups) {
+                gv[j] = ld_stream_f4(grad + 4 * gi);
+                rv[j] = ld_stream_f4(residual + 4 * gi);
+            } else {
+                float tg[4], tr[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int64_t e = 4 * gi + k;
+                    tg[k] = e < n ? ld_stream_f1(grad + e) : 0.0f;
+                    tr[k] = e < n ? ld_stream_f1(residual + e) : 0.0f;
+                }
+                gv[j] = make_float4(tg[0], tg[1], tg[2], tg[3]);
+                rv[j] = make_float4(tr[0], tr[1], tr[2], tr[3]);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < kTGroups; ++j) {
+            const int64_t gi = g0 + j * kWarp + lane;
+            float4 r = rv[j];
+            uint32_t c0 = tb_step(gv[j].x, r.x, neg, pos);
+            uint32_t c1 = tb_step(gv[j].y, r.y, neg, pos);
+            uint32_t c2 = tb_step(gv[j].z, r.z, neg, pos);
+            uint32_t c3 = tb_step(gv[j].w, r.w, neg, pos);
+            if (kVec && gi < full_groups) {
+                st_stream_f4(residual + 4 * gi, r);
+            } else {
+                const int64_t valid = n - 4 * gi;
+                const float rr[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    if (k < valid)
+                        st_stream_f1(residual + 4 * gi + k, rr[k]);
+                c0 = valid > 0 ? c0 : 0u;
+                c1 = valid > 1 ? c1 : 0u;
+                c2 = valid > 2 ? c2 : 0u;
+                c3 = valid > 3 ? c3 : 0u;
+            }
+            codes[j * kWarp + lane] = c0 | (c1 << 8) | (c2 << 16) | (c3 << 24);
+        }
+        __syncwarp();
+        uint32_t c[5];
+#pragma unroll
+        for (int i = 0; i < 5; ++i)
+            c[i] = codes[5 * lane + i];
+        const int64_t w = t * kWarp + lane;
+        if (w < nwords)
+            st_stream_u32(payload + w, pack_ternary_word(c));
+        __syncwarp();
+    }
+}
+
+// Byte -> (mask of its codes 01 in bits 4..0, mask of its codes 10 in bits
+// 9..5), element 5j + i of the byte at bit 4 - i.  Bytes above 242 never
+// occur in a record; they decode as if their digits were taken anyway.
+__device__ __forceinline__ void build_byte_table(uint16_t *table)
+{
+    for (int b = threadIdx.x; b < 256; b += blockDim.x) {
+        uint32_t v = (uint32_t)b, m01 = 0, m10 = 0;
+#pragma unroll
+        for (int i = 4; i >= 0; --i) {
+            const uint32_t d = v % 3u;
+            v /= 3u;
+            m01 |= (d == 1u ? 1u : 0u) << (4 - i);
+            m10 |= (d == 2u ? 1u : 0u) << (4 - i);
+        }
+        table[b] = (uint16_t)(m01 | (m10 << 5));
+    }
+}
+
+// The 01 / 10 masks of a payload word's 20 elements, element p at bit 19 - p.
+__device__ __forceinline__ void word_masks(const uint16_t *table, uint32_t word, uint32_t &is01,
+                                           uint32_t &is10)
+{
+    is01 = 0;
+    is10 = 0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const uint32_t m = table[(word >> (8 * k)) & 0xFFu];
+        is01 |= (m & 0x1Fu) << (15 - 5 * k);
+        is10 |= ((m >> 5) & 0x1Fu) << (15 - 5 * k);
+    }
+}
+
+struct RecordSet {
+    const uint32_t *rec[QGA_MAX_WORKERS];
+};
+
+// kMerge: sum of W records from +0 in worker order (skipping the exact +0
+// adds of code 00); otherwise W == 1 and each element is its code's value.
+template <bool kVec, bool kMerge>
+__global__ void __launch_bounds__(kThreads)
+    decode_ternary_kernel(const __grid_constant__ RecordSet set, int W, float *__restrict__ out,
+                          int64_t n)
+{
+    __shared__ uint16_t s_table[256];
+    __shared__ const uint32_t *s_payload[QGA_MAX_WORKERS];
+    __shared__ float s_neg[QGA_MAX_WORKERS], s_pos[QGA_MAX_WORKERS];
+    __shared__ float4 s_stage[kWarpsPerBlock][kWarp * 5];
+    build_byte_table(s_table);
+    if (threadIdx.x < W) {
+        const uint32_t *r = set.rec[threadIdx.x];
+        s_payload[threadIdx.x] = r + 3;
+        s_neg[threadIdx.x] = f32_from_bits(r[0]);
+        s_pos[threadIdx.x] = f32_from_bits(r[1]);
+    }
+    __syncthreads();
+    float4 *stage = s_stage[threadIdx.x >> 5];
+    const int lane = threadIdx.x & (kWarp - 1);
+    const int64_t nwords = (n + 19) / 20;
+    const int64_t tiles = (nwords + kWarp - 1) / kWarp;
+    for (int64_t t = warp_id(); t < tiles; t += warp_stride()) {
+        const int64_t w = t * kWarp + lane;
+        const bool ok = w < nwords;
+        float acc[20];
+#pragma unroll
+        for (int p = 0; p < 20; ++p)
+            acc[p] = 0.0f;
+        constexpr int kBatch = 8;
+        for (int wb = 0; wb < W; wb += kBatch) {
+            uint32_t words[kBatch];
+#pragma unroll
+            for (int i = 0; i < kBatch; ++i)
+                words[i] = (ok && wb + i < W) ? ld_stream_u32(s_payload[wb + i] + w) : 0u;
+#pragma unroll
+            for (int i = 0; i < kBatch; ++i) {
+                if (wb + i >= W) // warp-uniform
+                    break;
+                const float neg = s_neg[wb + i], pos = s_pos[wb + i];
+                uint32_t is01, is10;
+                word_masks(s_table, words[i], is01, is10);
+#pragma unroll
+                for (int p = 0; p < 20; ++p) {
+                    const uint32_t bit = 1u << (19 - p);
+                    if (kMerge) {
+                        if (is01 & bit)
+                            acc[p] = __fadd_rn(acc[p], pos);
+                        if (is10 & bit)
+                            acc[p] = __fadd_rn(acc[p], neg);
+                    } else {
+                        acc[p] = (is01 & bit) ? pos : ((is10 & bit) ? neg : 0.0f);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < 5; ++c)
+            stage[5 * lane + c] =
+                make_float4(acc[4 * c], acc[4 * c + 1], acc[4 * c + 2], acc[4 * c + 3]);
+        __syncwarp();
+#pragma unroll
+        for (int j = 0; j < 5; ++j) {
+            const int q = j * kWarp + lane; // group of 4 within the tile
+            store_group<kVec>(out, n, t * (kWarp * 5) + q, stage[q]);
+        }
+        __syncwarp();
+    }
+}
+
+std::atomic<int> occ_tq[2][64], occ_td[2][2][64];
+
+unsigned warps_grid(int64_t warp_items, int resident)
+{
+    return grid_for((warp_items + kWarpsPerBlock - 1) / kWarpsPerBlock, resident);
+}
+
+int launch_decode(const RecordSet &set, int W, float *out, int64_t n, cudaStream_t stream,
+                  bool merge)
+{
+    const int64_t tiles = ((n + 19) / 20 + kWarp - 1) / kWarp;
+    const bool vec = aligned(out, 16);
+    if (merge) {
+        if (vec) {
+            auto k = decode_ternary_kernel<true, true>;
+            k<<<warps_grid(tiles, resident_blocks(k, kThreads, occ_td[1][1])), kThreads, 0, stream>>>(set, W, out, n);
+        } else {
+            auto k = decode_ternary_kernel<false, true>;
+            k<<<warps_grid(tiles, resident_blocks(k, kThreads, occ_td[0][1])), kThreads, 0, stream>>>(set, W, out, n);
+        }
+    } else {
+        if (vec) {
+            auto k = decode_ternary_kernel<true, false>;
+            k<<<warps_grid(tiles, resident_blocks(k, kThreads, occ_td[1][0])), kThreads, 0, stream>>>(set, W, out, n);
+        } else {
+            auto k = decode_ternary_kernel<false, false>;
+            k<<<warps_grid(tiles, resident_blocks(k, kThreads, occ_td[0][0])), kThreads, 0, stream>>>(set, W, out, n);
+        }
+    }
+    return launch_status();
+}
+
+} // namespace
+} // namespace qga
+
+using namespace qga;
+
+extern "C" int64_t qga_ternary_words(int64_t n)
+{
+    if (n < 0)
+        return QGA_ERR_INVALID_ARG;
+    return 3 + (n + 19) / 20;
+}
+
+extern "C" int qga_quantize_ternary(const float *grad, float *residual, uint32_t *compr, int64_t n,
+                                    float neg_threshold, float pos_threshold, cudaStream_t stream)
+{
+    if (n < 0 || compr == nullptr || !aligned(compr, 4) || !finite_f32(neg_threshold) ||
+        !finite_f32(pos_threshold))
+        return QGA_ERR_INVALID_ARG;
+    if (n > 0 && (grad == nullptr || residual == nullptr || !aligned(grad, 4) || !aligned(residual, 4)))
+        return QGA_ERR_INVALID_ARG;
+    const int64_t tiles = (n + kTTileElems - 1) / kTTileElems;
+    if (aligned(grad, 16) && aligned(residual, 16)) {
+        auto k = quantize_ternary_kernel<true>;
+        k<<<warps_grid(tiles, resident_blocks(k, kThreads, occ_tq[1])), kThreads, 0, stream>>>(
+            grad, residual, compr, n, neg_threshold, pos_threshold);
+    } else {
+        auto k = quantize_ternary_kernel<false>;
+        k<<<warps_grid(tiles, resident_blocks(k, kThreads, occ_tq[0])), kThreads, 0, stream>>>(
+            grad, residual, compr, n, neg_threshold, pos_threshold);
+    }
+    return launch_status();
+}
+
+extern "C" int qga_dequantize_ternary(const uint32_t *compr, float *out, int64_t n,
+                                      cudaStream_t stream)
+{
+    if (n < 0 || compr == nullptr || !aligned(compr, 4))
+        return QGA_ERR_INVALID_ARG;
+    if (n == 0)
+        return QGA_OK;
+    if (out == nullptr || !aligned(out, 4))
+        return QGA_ERR_INVALID_ARG;
+    RecordSet set{};
+    set.rec[0] = compr;
+    return launch_decode(set, 1, out, n, stream, false);
+}
+
+extern "C" int qga_dequant_accumulate_ternary(const uint32_t *const *compr, int num_workers,
+                                              float *out, int64_t n, cudaStream_t stream)
+{
+    if (n < 0 || compr == nullptr || num_workers < 1 || num_workers > QGA_MAX_WORKERS)
+        return QGA_ERR_INVALID_ARG;
+    RecordSet set{};
+    for (int w = 0; w < num_workers; ++w) {
+        if (compr[w] == nullptr || !aligned(compr[w], 4))
+            return QGA_ERR_INVALID_ARG;
+        set.rec[w] = compr[w];
+    }
+    if (n == 0)
+        return QGA_OK;
+    if (out == nullptr || !aligned(out, 4))
+        return QGA_ERR_INVALID_ARG;
+    return launch_decode(set, num_workers, out, n, stream, true);
+}

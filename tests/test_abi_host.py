@@ -18,8 +18,8 @@ HEADER = os.path.join(ROOT, "include", "qga.h")
 
 @pytest.fixture(scope="module")
 def qga():
-    from quantized_gradient_aggregation_b200 import build
-    build.build()
+    import __graft_entry__
+    __graft_entry__._load_build_module().build()
     import quantized_gradient_aggregation_b200 as q
     return q
 
@@ -37,7 +37,8 @@ def test_header_declares_the_boundary():
                  "qga_quantize_2bit_bucket", "qga_dequant_accumulate_2bit_bucket",
                  "qga_qsgd_words", "qga_qsgd_mn_max", "qga_qsgd_mn_quantize",
                  "qga_qsgd_mn_dequant_accumulate", "qga_strerror", "qga_last_cuda_error",
-                 "qga_version"]:
+                 "qga_version", "qga_ternary_words", "qga_quantize_ternary",
+                 "qga_dequantize_ternary", "qga_dequant_accumulate_ternary"]:
         assert want in names, want
 
 
@@ -140,6 +141,14 @@ def test_invalid_arguments_are_rejected_before_any_cuda_call(qga):
     assert L.qga_qsgd_mn_dequant_accumulate(parr, 2, FAKE, 16, 5, None) == qga.QGA_ERR_UNSUPPORTED
     assert L.qga_qsgd_mn_dequant_accumulate(parr, 2, None, 16, 2, None) == E
     assert L.qga_qsgd_mn_dequant_accumulate(parr, 99, FAKE, 16, 2, None) == E
+    # dense ternary
+    assert L.qga_ternary_words(-1) == E and L.qga_ternary_words(0) == 3 and L.qga_ternary_words(21) == 5
+    assert L.qga_quantize_ternary(None, FAKE, FAKE, 16, -1.0, 1.0, None) == E
+    assert L.qga_quantize_ternary(FAKE, FAKE, FAKE, 16, nan, 1.0, None) == E
+    assert L.qga_quantize_ternary(FAKE + 1, FAKE, FAKE, 16, -1.0, 1.0, None) == E
+    assert L.qga_dequantize_ternary(FAKE, None, 16, None) == E
+    assert L.qga_dequant_accumulate_ternary(parr, 0, FAKE, 16, None) == E
+    assert L.qga_dequant_accumulate_ternary(parr, 2, FAKE + 2, 16, None) == E
     assert L.qga_last_cuda_error() == 0
 
 
