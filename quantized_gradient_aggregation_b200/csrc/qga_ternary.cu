@@ -19,9 +19,9 @@
 // loads: the stride of 5 words is odd) and forms each payload byte with one
 // byte-wise dot product against the weights 81, 27, 9, 3 (plus the fifth
 // code).  Decode geometry: a lane owns one payload word (20 elements); a
-// 243-entry shared table turns each byte into the bit masks of its codes
-// 01 and 10, and the outputs leave through a shared stage (again stride 5,
-// conflict-free) as coalesced 128-bit rows.
+// 256-entry shared table turns each byte into its five 2-bit codes or into
+// the bit masks of its codes 01 and 10, and the outputs leave through a
+// shared stage (again stride 5, conflict-free) as coalesced 128-bit rows.
 
 #include "qga_2bit_tiles.cuh"
 
@@ -128,20 +128,23 @@ __global__ void __launch_bounds__(kThreads)
 }
 
 // Byte -> (mask of its codes 01 in bits 4..0, mask of its codes 10 in bits
-// 9..5), element 5j + i of the byte at bit 4 - i.  Bytes above 242 never
-// occur in a record; they decode as if their digits were taken anyway.
-__device__ __forceinline__ void build_byte_table(uint16_t *table)
+// 9..5), element 5j + i of the byte at bit 4 - i; and byte -> its five 2-bit
+// codes, element 5j + i in bits 9 - 2i .. 8 - 2i.  Digits are taken mod 3
+// (bytes above 242 never occur in a record).
+__device__ __forceinline__ void build_byte_tables(uint16_t *masks, uint16_t *codes)
 {
     for (int b = threadIdx.x; b < 256; b += blockDim.x) {
-        uint32_t v = (uint32_t)b, m01 = 0, m10 = 0;
+        uint32_t v = (uint32_t)b, m01 = 0, m10 = 0, c = 0;
 #pragma unroll
         for (int i = 4; i >= 0; --i) {
             const uint32_t d = v % 3u;
             v /= 3u;
             m01 |= (d == 1u ? 1u : 0u) << (4 - i);
             m10 |= (d == 2u ? 1u : 0u) << (4 - i);
+            c |= (d & 3u) << (2 * (4 - i));
         }
-        table[b] = (uint16_t)(m01 | (m10 << 5));
+        masks[b] = (uint16_t)(m01 | (m10 << 5));
+        codes[b] = (uint16_t)c;
     }
 }
 
@@ -163,24 +166,33 @@ struct RecordSet {
     const uint32_t *rec[QGA_MAX_WORKERS];
 };
 
-// kMerge: sum of W records from +0 in worker order (skipping the exact +0
-// adds of code 00); otherwise W == 1 and each element is its code's value.
+// kMerge: sum of W records from +0 in worker order (bit for bit the 2-bit
+// merge's sums); otherwise W == 1 and each element is its code's value.
+// As in the 2-bit merge, even workers go through a per-worker pair table
+// (shared loads + paired adds) and odd workers through code masks and
+// predicated adds (skipping the exact +0 adds of code 00), so that neither
+// the integer pipe nor the load/store pipe saturates alone.
 template <bool kVec, bool kMerge>
 __global__ void __launch_bounds__(kThreads)
     decode_ternary_kernel(const __grid_constant__ RecordSet set, int W, float *__restrict__ out,
                           int64_t n)
 {
-    __shared__ uint16_t s_table[256];
+    __shared__ uint16_t s_masks[256], s_codes[256];
     __shared__ const uint32_t *s_payload[QGA_MAX_WORKERS];
     __shared__ float s_neg[QGA_MAX_WORKERS], s_pos[QGA_MAX_WORKERS];
+    __shared__ float2 s_pair[kMerge ? QGA_MAX_WORKERS : 1][16];
     __shared__ float4 s_stage[kWarpsPerBlock][kWarp * 5];
-    build_byte_table(s_table);
+    build_byte_tables(s_masks, s_codes);
     if (threadIdx.x < W) {
         const uint32_t *r = set.rec[threadIdx.x];
         s_payload[threadIdx.x] = r + 3;
         s_neg[threadIdx.x] = f32_from_bits(r[0]);
         s_pos[threadIdx.x] = f32_from_bits(r[1]);
     }
+    __syncthreads();
+    if (kMerge)
+        for (int i = threadIdx.x; i < W * 16; i += kThreads)
+            s_pair[i >> 4][i & 15] = pair_entry(i & 15, s_neg[i >> 4], s_pos[i >> 4]);
     __syncthreads();
     float4 *stage = s_stage[threadIdx.x >> 5];
     const int lane = threadIdx.x & (kWarp - 1);
@@ -189,10 +201,10 @@ __global__ void __launch_bounds__(kThreads)
     for (int64_t t = warp_id(); t < tiles; t += warp_stride()) {
         const int64_t w = t * kWarp + lane;
         const bool ok = w < nwords;
-        float acc[20];
+        float2 acc[10];
 #pragma unroll
-        for (int p = 0; p < 20; ++p)
-            acc[p] = 0.0f;
+        for (int q = 0; q < 10; ++q)
+            acc[q] = make_float2(0.0f, 0.0f);
         constexpr int kBatch = 8;
         for (int wb = 0; wb < W; wb += kBatch) {
             uint32_t words[kBatch];
@@ -203,27 +215,46 @@ __global__ void __launch_bounds__(kThreads)
             for (int i = 0; i < kBatch; ++i) {
                 if (wb + i >= W) // warp-uniform
                     break;
-                const float neg = s_neg[wb + i], pos = s_pos[wb + i];
-                uint32_t is01, is10;
-                word_masks(s_table, words[i], is01, is10);
+                const uint32_t word = words[i];
+                if (kMerge && (i & 1) == 0) {
+                    // the 20 codes as a 40-bit string, element 0 in bits 39..38
+                    const uint32_t c0 = s_codes[word & 0xFFu], c1 = s_codes[(word >> 8) & 0xFFu];
+                    const uint32_t c2 = s_codes[(word >> 16) & 0xFFu], c3 = s_codes[word >> 24];
+                    const uint32_t hi = c0 >> 2;
+                    const uint32_t lo = (c0 << 30) | (c1 << 20) | (c2 << 10) | c3;
+                    const char *tb = reinterpret_cast<const char *>(s_pair[wb + i]);
 #pragma unroll
-                for (int p = 0; p < 20; ++p) {
-                    const uint32_t bit = 1u << (19 - p);
-                    if (kMerge) {
-                        if (is01 & bit)
-                            acc[p] = __fadd_rn(acc[p], pos);
-                        if (is10 & bit)
-                            acc[p] = __fadd_rn(acc[p], neg);
-                    } else {
-                        acc[p] = (is01 & bit) ? pos : ((is10 & bit) ? neg : 0.0f);
+                    for (int q = 0; q < 10; ++q) {
+                        // 4 code bits of elements 2q, 2q+1, times the 8-byte entry size
+                        const int sh = 36 - 4 * q;
+                        const uint32_t nib = sh >= 32 ? (hi >> (sh - 32)) : (lo >> sh);
+                        const uint32_t off = (nib & 0xFu) << 3;
+                        acc[q] = __fadd2_rn(acc[q], *reinterpret_cast<const float2 *>(tb + off));
+                    }
+                } else {
+                    const float neg = s_neg[wb + i], pos = s_pos[wb + i];
+                    uint32_t is01, is10;
+                    word_masks(s_masks, word, is01, is10);
+#pragma unroll
+                    for (int p = 0; p < 20; ++p) {
+                        const uint32_t bit = 1u << (19 - p);
+                        float &a = (p & 1) ? acc[p >> 1].y : acc[p >> 1].x;
+                        if (kMerge) {
+                            if (is01 & bit)
+                                a = __fadd_rn(a, pos);
+                            if (is10 & bit)
+                                a = __fadd_rn(a, neg);
+                        } else {
+                            a = (is01 & bit) ? pos : ((is10 & bit) ? neg : 0.0f);
+                        }
                     }
                 }
             }
         }
 #pragma unroll
         for (int c = 0; c < 5; ++c)
-            stage[5 * lane + c] =
-                make_float4(acc[4 * c], acc[4 * c + 1], acc[4 * c + 2], acc[4 * c + 3]);
+            stage[5 * lane + c] = make_float4(acc[2 * c].x, acc[2 * c].y, acc[2 * c + 1].x,
+                                              acc[2 * c + 1].y);
         __syncwarp();
 #pragma unroll
         for (int j = 0; j < 5; ++j) {
