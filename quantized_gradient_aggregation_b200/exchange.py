@@ -1,0 +1,70 @@
+"""Data-parallel exchange of compressed gradients across ranks.
+
+The receiver-side merge of MXNet pull request #8342 "[WIP] 2bit gradient
+compression" ("Local kvstore": every device quantizes its gradient, the
+compressed arrays travel to the device that reduces, which dequantizes and
+sums them), made symmetric for one process per GPU: every rank quantizes
+its own gradient with error feedback, the W records are all-gathered into
+one contiguous buffer (NCCL over NVLink / NVSwitch; a record is 1/16 of the
+fp32 gradient), and every rank merges the same W records in rank order, so
+all ranks hold the same aggregate bit for bit without a second exchange.
+The gathered buffer holds W records of ``words`` int32 each, rank r's record
+in row r.
+
+Every arithmetic step runs in the library's CUDA kernels; this module only
+orders them around one collective on the current stream.
+"""
+from __future__ import annotations
+
+import torch
+import torch.distributed as dist
+
+from . import (qga_2bit_words, qga_dequant_accumulate_2bit, qga_dequant_accumulate_ternary,
+               qga_quantize_2bit, qga_quantize_ternary, qga_ternary_words)
+
+_FORMATS = {
+    "2bit": (qga_2bit_words, qga_quantize_2bit, qga_dequant_accumulate_2bit),
+    "ternary": (qga_ternary_words, qga_quantize_ternary, qga_dequant_accumulate_ternary),
+}
+
+
+def gather_records(local: torch.Tensor, gathered: torch.Tensor, group=None):
+    """All-gather one record per rank into ``gathered`` (world * words
+    int32) and return its rows, row r = rank r's record."""
+    world = dist.get_world_size(group)
+    words = local.numel()
+    if gathered.numel() != world * words:
+        raise ValueError(f"gathered holds {gathered.numel()} words, need {world} x {words}")
+    dist.all_gather_into_tensor(gathered, local, group=group)
+    return list(gathered.view(world, words).unbind(0))
+
+
+class CompressedAllGather:
+    """One compressed all-gather step for an n-element gradient.
+
+    ``step(grad, residual, out)`` quantizes ``grad`` against ``residual``
+    (updated in place) with the thresholds given here, all-gathers the
+    records of the ``group``'s ranks and writes their merge (worker order =
+    rank order) into ``out``.  The two record buffers are allocated once,
+    here, on the current CUDA device.
+    """
+
+    def __init__(self, n: int, neg_threshold: float, pos_threshold: float, group=None,
+                 fmt: str = "2bit"):
+        if fmt not in _FORMATS:
+            raise ValueError(f"format {fmt!r}: one of {sorted(_FORMATS)}")
+        self.n = int(n)
+        self.neg = float(neg_threshold)
+        self.pos = float(pos_threshold)
+        self.group = group
+        self.world = dist.get_world_size(group)
+        words_fn, self._quantize, self._merge = _FORMATS[fmt]
+        self.words = int(words_fn(self.n))
+        device = torch.device("cuda", torch.cuda.current_device())
+        self.local = torch.empty(self.words, dtype=torch.int32, device=device)
+        self.gathered = torch.empty(self.world * self.words, dtype=torch.int32, device=device)
+
+    def step(self, grad: torch.Tensor, residual: torch.Tensor, out: torch.Tensor) -> None:
+        self._quantize(grad, residual, self.local, self.neg, self.pos)
+        records = gather_records(self.local, self.gathered, self.group)
+        self._merge(records, out)

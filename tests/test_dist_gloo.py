@@ -89,3 +89,24 @@ def test_reference_arm_runs_on_rank_zero_only():
     assert line["impl"] == "reference" and line["n_gpus"] == 2
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
     assert outs[1].strip() == ""
+
+
+def test_record_gather_layout_on_two_and_three_ranks():
+    """The exchange's gather step: every rank ends up with the same buffer,
+    rank r's record in row r (the merge then adds the rows in rank order).
+    The records here are synthetic words, so no GPU is needed."""
+    for world in (2, 3):
+        outs = _run_ranks("""
+            import torch, hashlib
+            from quantized_gradient_aggregation_b200.exchange import gather_records
+            words = 37
+            local = torch.arange(words, dtype=torch.int32) * 1000 + rank
+            gathered = torch.empty(world * words, dtype=torch.int32)
+            rows = gather_records(local, gathered)
+            assert len(rows) == world
+            for r, row in enumerate(rows):
+                assert row.tolist() == [w * 1000 + r for w in range(words)], r
+            print(hashlib.sha256(gathered.numpy().tobytes()).hexdigest())
+        """, world=world)
+        digests = {o.strip().splitlines()[-1] for o in outs}
+        assert len(digests) == 1
