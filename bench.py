@@ -530,39 +530,62 @@ def time_rows(dev, stream, peak, reps=20):
 
 def run_e2e(args, w, dev_grads, res, comprs, out, quant, merge, stream, world, dev):
     """Same step with the gradients arriving from pinned host memory and the
-    aggregate read back, copies inside the timed region."""
+    aggregate read back, copies inside the timed region.  Copies run on a
+    second stream: worker k's upload overlaps the quantize of worker k - 1,
+    and the aggregate's download (the other PCIe direction) overlaps the
+    next step's uploads; events order every reuse of a buffer."""
     import torch
-    import torch.distributed as dist
     n, W = w.n, w.workers
     host = [torch.empty(n, dtype=torch.float32, pin_memory=True) for _ in range(W)]
     for k in range(W):
         host[k].copy_(dev_grads[k], non_blocking=False)
     host_out = torch.empty(n, dtype=torch.float32, pin_memory=True)
+    copy_stream = torch.cuda.Stream(device=dev)
     K = max(3, min(args.steps, 10))
+    landed = [torch.cuda.Event() for _ in range(W)]
+    consumed = [torch.cuda.Event() for _ in range(W)]
+    merged = torch.cuda.Event()
+    downloaded = torch.cuda.Event()
+    for e in consumed:
+        e.record(stream)
+    downloaded.record(stream)
 
     def step():
         for k in range(W):
-            dev_grads[k].copy_(host[k], non_blocking=True)
+            with torch.cuda.stream(copy_stream):
+                copy_stream.wait_event(consumed[k])      # previous quantize of worker k is done
+                dev_grads[k].copy_(host[k], non_blocking=True)
+                landed[k].record(copy_stream)
+            stream.wait_event(landed[k])
             quant(0, k)
+            consumed[k].record(stream)
+        stream.wait_event(downloaded)                    # previous aggregate has left the device
         merge()
-        host_out.copy_(out, non_blocking=True)
+        merged.record(stream)
+        with torch.cuda.stream(copy_stream):
+            copy_stream.wait_event(merged)
+            host_out.copy_(out, non_blocking=True)
+            downloaded.record(copy_stream)
 
     for _ in range(2):
         step()
     torch.cuda.synchronize()
     if world > 1:
+        import torch.distributed as dist
         dist.barrier()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
+    copy_stream.wait_event(a)
     for _ in range(K):
         step()
+    stream.wait_event(downloaded)
     b.record(stream)
     torch.cuda.synchronize()
     (ms,) = max_over_ranks([a.elapsed_time(b)], world, dev)
     return {"value": job_gelem_per_s(world, W, n, K, ms), "unit": "Gelem/s",
             "h2d_bytes_per_step": W * n * 4, "d2h_bytes_per_step": n * 4, "steps": K,
-            "path": "pinned host gradients -> cudaMemcpyAsync -> qga_quantize_2bit x8 -> "
-                    "qga_dequant_accumulate_2bit -> pinned host aggregate"}
+            "path": "pinned host gradients -> cudaMemcpyAsync (copy stream) -> qga_quantize_2bit x8 "
+                    "-> qga_dequant_accumulate_2bit -> pinned host aggregate (copy stream)"}
 
 
 def main():
