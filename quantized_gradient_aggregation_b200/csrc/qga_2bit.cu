@@ -57,8 +57,12 @@ struct RecordSet {
 
 // kW > 0: compiled for exactly kW workers (record pointers and loop bounds
 // are constants); kW == 0: any W up to QGA_MAX_WORKERS.
+#ifndef QGA_MERGE_MIN_BLOCKS
+#define QGA_MERGE_MIN_BLOCKS 4
+#endif
+
 template <bool kVec, int kW>
-__global__ void __launch_bounds__(kThreads, 4)
+__global__ void __launch_bounds__(kThreads, QGA_MERGE_MIN_BLOCKS)
     dequant_accumulate_2bit_kernel(const __grid_constant__ RecordSet set, int W,
                                    float *__restrict__ out, int64_t n)
 {

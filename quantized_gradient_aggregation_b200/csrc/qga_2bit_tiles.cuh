@@ -237,7 +237,10 @@ __device__ __forceinline__ void dequantize_2bit_tile(const uint32_t *__restrict_
 // through a per-warp shared-memory stage (xor-swizzled so that both the
 // 128-bit writes and the 128-bit reads are free of bank conflicts) as fully
 // coalesced 128-bit rows.
-constexpr int kMergeSlots = 2;                         // words per lane per slice
+#ifndef QGA_MERGE_SLOTS
+#define QGA_MERGE_SLOTS 2
+#endif
+constexpr int kMergeSlots = QGA_MERGE_SLOTS;           // words per lane per slice
 constexpr int kSliceWords = kWarp * kMergeSlots;       // 64
 constexpr int64_t kSliceElems = kSliceWords * 16;      // 1024
 constexpr int kStagePerWarp = kSliceWords * 4;         // float4 per warp (4 KB)
