@@ -38,14 +38,6 @@ def build(force: bool = False) -> str:
     return _LIB
 
 
-def _u32p(a):
-    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_uint32))
-
-
-def _f32p(a):
-    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_float))
-
-
 def _ptr_array(arrays):
     arr = (ctypes.c_void_p * max(1, len(arrays)))()
     for i, a in enumerate(arrays):

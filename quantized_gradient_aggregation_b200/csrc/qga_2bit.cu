@@ -7,9 +7,12 @@
 // (the receiver dequantizes every worker's gradient and sums them).
 //
 // Each kernel is one pass over HBM with a persistent grid (every SM filled
-// once; warps stride over 512-element tiles).  Nothing is filled or cleared
-// by a separate launch: the quantize kernel writes every payload word
-// (including the zero tail codes) and its block 0 writes the header.
+// once; warps stride over tiles: 512 elements for an fp32 quantize or a
+// dequantize, 1024 for a bf16 quantize or a merge slice).  Nothing is filled
+// or cleared by a separate launch: the quantize kernel writes every payload
+// word (including the zero tail codes) and its block 0 writes the header.
+// The merge's occupancy and words per lane are build-time settings
+// (QGA_MERGE_MIN_BLOCKS, QGA_MERGE_SLOTS); the defaults are the measured best.
 
 #include "qga_2bit_tiles.cuh"
 

@@ -10,7 +10,7 @@ import torch
 import torch.distributed as dist
 
 import oracle
-from gpu_util import DEV, f32, qga, same_bits_f32
+from gpu_util import DEV, f32, same_bits_f32
 
 pytestmark = pytest.mark.gpu
 
