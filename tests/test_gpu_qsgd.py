@@ -202,7 +202,8 @@ def test_quantize_levels_next_to_integer_boundaries(b):
     seed = 987654321
     n = 4096
     rng = np.random.default_rng(b)
-    deltas = np.array([1e-7, -1e-7, 3e-6, -3e-6, 2e-5, -2e-5, 4e-5, -4e-5, 6e-5, -6e-5, 1e-4, -2e-4])
+    deltas = np.array([1e-7, -1e-7, 3e-6, -3e-6, 2e-5, -2e-5, 4e-5, -4e-5, 6e-5, -6e-5, 1e-4, -2e-4,
+                       1.3e-4, -1.3e-4, 1.5e-4, -1.5e-4, 3e-4, -3e-4])
     g = np.empty(n, np.float32)
     for e in range(n):
         u = oracle.qsgd_uniform(seed, e)
@@ -215,4 +216,24 @@ def test_quantize_levels_next_to_integer_boundaries(b):
     c = torch.empty(q.qga_qsgd_words(n, b), dtype=torch.int32, device=DEV)
     q.qga_qsgd_mn_quantize(dev_g, c, b, seed, Md)
     want = oracle.qsgd_mn_quantize(g, b, seed, M)
+    assert np.array_equal(u32(c), want), first_diff(u32(c), want)
+
+
+@pytest.mark.parametrize("b", BITS)
+def test_quantize_16M_full(b):
+    """Every code of 2^24 elements spread over all levels (|g| uniform up to
+    M, both signs) against the oracle."""
+    q = qga()
+    n = 1 << 24
+    gen = torch.Generator(device=DEV)
+    gen.manual_seed(1000 + b)
+    g = (torch.rand(n, device=DEV, generator=gen) * 2 - 1) * 6.0
+    M = torch.empty(1, device=DEV)
+    q.qga_qsgd_mn_max([g], M)
+    g_host = f32(g)
+    M_or = oracle.qsgd_mn_max([g_host])
+    assert M.item() == M_or
+    c = torch.empty(q.qga_qsgd_words(n, b), dtype=torch.int32, device=DEV)
+    q.qga_qsgd_mn_quantize(g, c, b, 2024 + b, M)
+    want = oracle.qsgd_mn_quantize(g_host, b, 2024 + b, M_or)
     assert np.array_equal(u32(c), want), first_diff(u32(c), want)
