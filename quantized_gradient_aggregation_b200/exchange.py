@@ -68,3 +68,56 @@ class CompressedAllGather:
         self._quantize(grad, residual, self.local, self.neg, self.pos)
         records = gather_records(self.local, self.gathered, self.group)
         self._merge(records, out)
+
+
+class BucketedCompressedAllGather:
+    """The exchange over a list of buckets (each a list of tensors quantized
+    by one bucket launch), pipelined: bucket b's records are all-gathered by
+    NCCL while the current stream already quantizes bucket b + 1, and each
+    bucket's merge waits only for its own all-gather.
+
+    ``buckets``: per bucket, the tensor sizes; ``neg`` / ``pos``: per bucket,
+    per-tensor thresholds.  ``step(grads, residuals, outs)`` takes per bucket
+    the gradient tensors (fp32 or bf16, one dtype per bucket), the fp32
+    residuals (updated in place) and one flat fp32 output holding the
+    bucket's merged tensors one after the other.
+    """
+
+    def __init__(self, buckets, neg, pos, group=None):
+        from . import qga_2bit_bucket_words
+        self.sizes = [list(map(int, b)) for b in buckets]
+        self.neg = [list(map(float, x)) for x in neg]
+        self.pos = [list(map(float, x)) for x in pos]
+        self.group = group
+        self.world = dist.get_world_size(group)
+        device = torch.device("cuda", torch.cuda.current_device())
+        self.words = [qga_2bit_bucket_words(s) for s in self.sizes]
+        self.local = [torch.empty(w, dtype=torch.int32, device=device) for w in self.words]
+        self.gathered = [torch.empty(self.world * w, dtype=torch.int32, device=device)
+                         for w in self.words]
+        self._tables = None
+        self._table_key = None
+
+    def records(self, b):
+        return list(self.gathered[b].view(self.world, self.words[b]).unbind(0))
+
+    def step(self, grads, residuals, outs) -> None:
+        from . import (make_bucket_table, qga_dequant_accumulate_2bit_bucket,
+                       qga_quantize_2bit_bucket)
+        key = tuple((g.data_ptr(), r.data_ptr()) for bg, br in zip(grads, residuals)
+                    for g, r in zip(bg, br))
+        if key != self._table_key:  # descriptor tables: rebuilt only when a buffer moved
+            self._tables = [make_bucket_table(grads[b], residuals[b], self.neg[b], self.pos[b])
+                            for b in range(len(self.sizes))]
+            self._table_key = key
+        works = []
+        for b in range(len(self.sizes)):
+            qga_quantize_2bit_bucket(grads[b], residuals[b], self.neg[b], self.pos[b],
+                                     self.local[b], table=self._tables[b])
+            # NCCL orders the collective after the work already on the current
+            # stream, and runs it beside the next bucket's quantize
+            works.append(dist.all_gather_into_tensor(self.gathered[b], self.local[b],
+                                                     group=self.group, async_op=True))
+        for b, work in enumerate(works):
+            work.wait()  # the current stream waits for bucket b's records only
+            qga_dequant_accumulate_2bit_bucket(self.records(b), self.sizes[b], outs[b])

@@ -50,3 +50,30 @@ def test_exchange_one_rank(nccl_group, fmt):
         assert np.array_equal(ex.gathered.cpu().numpy().view(np.uint32), rec), it
         assert same_bits_f32(f32(r), r_host), it
         assert same_bits_f32(f32(out), want), it
+
+
+def test_bucketed_exchange_one_rank(nccl_group):
+    """Two BERT-like buckets (bf16 gradients), pipelined all-gathers, three
+    steps with carried residuals, against the oracle's bucket functions."""
+    from quantized_gradient_aggregation_b200.exchange import BucketedCompressedAllGather
+    buckets = [[768, 3072, 589_824, 17], [30_000, 5, 768 * 16]]
+    neg = [[-2e-3] * len(b) for b in buckets]
+    pos = [[2e-3 + 1e-4 * i for i in range(len(b))] for b in buckets]
+    gen = torch.Generator(device=DEV)
+    gen.manual_seed(12)
+    grads = [[(torch.randn(s, device=DEV, generator=gen) * 1e-3).to(torch.bfloat16) for s in b]
+             for b in buckets]
+    res = [[torch.zeros(s, device=DEV) for s in b] for b in buckets]
+    outs = [torch.empty(sum(b), device=DEV) for b in buckets]
+    ex = BucketedCompressedAllGather(buckets, neg, pos)
+    g_host = [[g.cpu().view(torch.int16).numpy().view(np.uint16) for g in b] for b in grads]
+    r_host = [[np.zeros(s, np.float32) for s in b] for b in buckets]
+    for it in range(3):
+        ex.step(grads, res, outs)
+        for b in range(len(buckets)):
+            want_c, r_host[b] = oracle.quantize_2bit_bucket(g_host[b], r_host[b], neg[b], pos[b])
+            assert np.array_equal(ex.gathered[b].cpu().numpy().view(np.uint32), want_c), (it, b)
+            want = oracle.dequant_accumulate_2bit_bucket([want_c], buckets[b])
+            assert same_bits_f32(f32(outs[b]), want), (it, b)
+            for t in range(len(buckets[b])):
+                assert same_bits_f32(f32(res[b][t]), r_host[b][t]), (it, b, t)
