@@ -1,7 +1,9 @@
 """The library calls are stream-ordered, never synchronize and never
 allocate: a whole step (W quantizes + the merge; the bucket path; the QSGD
-path with its memset) captures into a CUDA graph, and replaying the graph
-gives the same bits as running the calls eagerly on the same inputs."""
+path with its memset) captures into a CUDA graph -- torch captures in the
+"global" error mode, where a device allocation or a synchronizing call from
+any thread aborts the capture -- and replaying the graph gives the same bits
+as running the calls eagerly on the same inputs."""
 import numpy as np
 import pytest
 import torch
@@ -28,24 +30,26 @@ def test_two_bit_step_in_a_cuda_graph():
     gen.manual_seed(8)
     grads = [torch.randn(n, device=DEV, generator=gen) for _ in range(W)]
     res0 = [torch.rand(n, device=DEV, generator=gen) - 0.5 for _ in range(W)]
-    # eager: three steps
+    # eager: three steps; the device's free memory does not move
     res_e = [r.clone() for r in res0]
     comprs_e = [torch.empty(q.qga_2bit_words(n), dtype=torch.int32, device=DEV) for _ in range(W)]
     out_e = torch.empty(n, device=DEV)
+    torch.cuda.synchronize()
+    free_before, _ = torch.cuda.mem_get_info()
     for _ in range(3):
         _step_2bit(q, grads, res_e, comprs_e, out_e)
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free_before, "a library call allocated device memory"
     # graph: capture one step, replay three times
     res_g = [r.clone() for r in res0]
     comprs_g = [torch.empty_like(c) for c in comprs_e]
     out_g = torch.empty(n, device=DEV)
     torch.cuda.synchronize()
-    before = torch.cuda.memory_allocated()
     graph = torch.cuda.CUDAGraph()
     side = torch.cuda.Stream()
     with torch.cuda.stream(side):
         with torch.cuda.graph(graph, stream=side):
             _step_2bit(q, grads, res_g, comprs_g, out_g)
-    assert torch.cuda.memory_allocated() == before, "a library call allocated device memory"
     # capture does not execute: the residuals are still the initial ones
     assert all(np.array_equal(a, b) for a, b in zip(_bits(res_g), _bits(res0)))
     for _ in range(3):
