@@ -46,7 +46,7 @@ FALLBACK_HBM_GBS = 6650.0
 # launch of the quantize kernel (profiles/quantize_2bit_kernel_fp32_vgg16.md),
 # keyed by the hash of the sources that kernel is compiled from; reported as
 # null once they have changed since the capture.
-MEASURED_TRAFFIC = {"1b60ae20dff0ea9c": 11.905}   # 1.6469 GB per launch of n = 138,357,544
+MEASURED_TRAFFIC = {"7c5c6e8e1703be24": 11.905}   # 1.6471 GB per launch of n = 138,357,544
 QUANT_SOURCES = ("qga_common.cuh", "qga_2bit_tiles.cuh", "qga_2bit.cu")
 
 
@@ -63,6 +63,8 @@ def parse_args():
     # smaller cases of the same step, for profiler captures (not bench lines)
     p.add_argument("--n", type=int, default=None, help="elements per worker (default: workload n)")
     p.add_argument("--iterations", type=int, default=None, help="resident gradient sets")
+    p.add_argument("--rows-scale", type=int, default=1,
+                   help="divide the per-row workloads' sizes by this (profiler captures)")
     return p.parse_args()
 
 
@@ -266,7 +268,7 @@ def run_qga(args, rank, world, local_rank):
     if args.n is not None or args.iterations is not None:
         import dataclasses
         w = dataclasses.replace(w, n=args.n or w.n, iterations=args.iterations or w.iterations,
-                                name=w.name + "-small")
+                                name=w.name + "-reduced")
     n, W, iters = w.n, w.workers, w.iterations
     L = q.lib()
 
@@ -339,7 +341,8 @@ def run_qga(args, rank, world, local_rank):
                                            stream, world, dev)
     del grads, res, comprs, out
     torch.cuda.empty_cache()
-    rows = None if args.no_rows else time_rows(dev, stream, measured_peaks()[0])
+    rows = None if args.no_rows else time_rows(dev, stream, measured_peaks()[0],
+                                               scale=max(1, args.rows_scale))
 
     if rank != 0:
         return
@@ -411,9 +414,10 @@ def _row(seconds, elems, bytes_per_elem, peak, launches, **extra):
     return d
 
 
-def time_rows(dev, stream, peak, reps=20):
+def time_rows(dev, stream, peak, reps=20, scale=1):
     """Device time of every other row of the hot path, each on its own
-    workload at full size (inputs resident, larger than L2)."""
+    workload at full size (inputs resident, larger than L2); ``scale`` > 1
+    shrinks the flat workloads for profiler captures only."""
     import torch
 
     import quantized_gradient_aggregation_b200 as q
@@ -429,15 +433,15 @@ def time_rows(dev, stream, peak, reps=20):
 
     # dequantize of one VGG16-sized record
     w = workloads.WORKLOADS[WORKLOAD]
-    n = w.n
-    g = workloads.gradient(w, 0, 0, device=dev)
+    n = w.n // scale
+    g = workloads.gradient(w, 0, 0, device=dev, n=n)
     r = torch.zeros(n, device=dev)
     c = torch.empty(q.qga_2bit_words(n), dtype=torch.int32, device=dev)
     q.qga_quantize_2bit(g, r, c, w.neg_thr, w.pos_thr)
     out = torch.empty(n, device=dev)
     t = _time_launches(stream, lambda: ok(L.qga_dequantize_2bit(vp(c.data_ptr()), vp(out.data_ptr()),
                                                                 n, sp), "dequantize"), reps)
-    rows["dequantize_2bit"] = _row(t, n, 4.25, peak, reps + 3, workload="vgg16 record, n=138,357,544")
+    rows["dequantize_2bit"] = _row(t, n, 4.25, peak, reps + 3, workload=f"vgg16 record, n={n:,}")
     del c
 
     # dense ternary records (5 codes per byte): quantize and the 8-worker merge
@@ -445,7 +449,7 @@ def time_rows(dev, stream, peak, reps=20):
     t = _time_launches(stream, lambda: ok(L.qga_quantize_ternary(
         vp(g.data_ptr()), vp(r.data_ptr()), vp(ct[0].data_ptr()), n, w.neg_thr, w.pos_thr, sp),
         "quantize_ternary"), reps)
-    rows["quantize_ternary"] = _row(t, n, 12.2, peak, reps + 3, workload="vgg16 gradient, n=138,357,544")
+    rows["quantize_ternary"] = _row(t, n, 12.2, peak, reps + 3, workload=f"vgg16 gradient, n={n:,}")
     for k in range(1, w.workers):
         ct[k].copy_(ct[0])
     tarr = (ctypes.c_void_p * w.workers)(*[cc.data_ptr() for cc in ct])
@@ -453,7 +457,7 @@ def time_rows(dev, stream, peak, reps=20):
     t = _time_launches(stream, lambda: ok(L.qga_dequant_accumulate_ternary(
         tp, w.workers, vp(out.data_ptr()), n, sp), "merge_ternary"), reps)
     rows["dequant_accumulate_ternary_w8"] = _row(t, n, 0.2 * w.workers + 4, peak, reps + 3,
-                                                 workload="8 dense records of n=138,357,544")
+                                                 workload=f"8 dense records of n={n:,}")
     del g, r, out, ct
 
     # BERT-Base bucket: quantize (bf16 grad) and 4-worker merge
@@ -494,15 +498,15 @@ def time_rows(dev, stream, peak, reps=20):
 
     # QSGD-MaxNorm: max over 8 workers, quantize per b, merge of 8
     wq = workloads.WORKLOADS["qsgd-128M-8w"]
-    nq, Wq = wq.n, wq.workers
-    grads = [workloads.gradient(wq, k, 0, device=dev) for k in range(Wq)]
+    nq, Wq = wq.n // scale, wq.workers
+    grads = [workloads.gradient(wq, k, 0, device=dev, n=nq) for k in range(Wq)]
     M = torch.empty(1, device=dev)
     garr = (ctypes.c_void_p * Wq)(*[gg.data_ptr() for gg in grads])
     gp = ctypes.cast(garr, ctypes.POINTER(ctypes.c_void_p))
     t = _time_launches(stream, lambda: ok(L.qga_qsgd_mn_max(gp, Wq, nq, vp(M.data_ptr()), sp),
                                           "qsgd_max"), reps)
     rows["qsgd_mn_max_w8"] = _row(t, nq * Wq, 4.0, peak, reps + 3,
-                                  workload="8 x 2^27 fp32 (0.1% outliers of 50)")
+                                  workload=f"8 x {nq:,} fp32 (0.1% outliers of 50)")
     out = torch.empty(nq, device=dev)
     for b in wq.bits:
         cq = [torch.empty(q.qga_qsgd_words(nq, b), dtype=torch.int32, device=dev) for _ in range(Wq)]
@@ -515,14 +519,15 @@ def time_rows(dev, stream, peak, reps=20):
             quant_q(k)
         t = _time_launches(stream, quant_q, reps)
         rows[f"qsgd_mn_quantize_b{b}"] = _row(t, nq, 4 + b / 8, peak, reps + 3 + Wq,
-                                              workload=f"2^27 fp32, b={b}")
+                                              workload=f"{nq:,} fp32, b={b}")
         carr = (ctypes.c_void_p * Wq)(*[cc.data_ptr() for cc in cq])
         cp = ctypes.cast(carr, ctypes.POINTER(ctypes.c_void_p))
         t = _time_launches(stream, lambda: ok(L.qga_qsgd_mn_dequant_accumulate(
             cp, Wq, vp(out.data_ptr()), nq, b, sp), "qsgd_merge"), reps)
         rows[f"qsgd_mn_dequant_accumulate_b{b}_w8"] = _row(t, nq, Wq * b / 8 + 4, peak, reps + 3,
-                                                          workload=f"8 records of 2^27, b={b}")
+                                                          workload=f"8 records of {nq:,}, b={b}")
         del cq
+
     del grads, out
     torch.cuda.empty_cache()
     return rows
