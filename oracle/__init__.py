@@ -81,6 +81,10 @@ def _declare(L):
     L.oracle_qsgd_mn_quantize.argtypes = [vp, vp, i64, i32, u64, f32]
     L.oracle_qsgd_mn_dequant_accumulate.argtypes = [vp, i32, vp, i64, i32]
     L.oracle_ternary_words.restype = i64
+    L.oracle_grandk_mn_max.restype = f32
+    L.oracle_grandk_mn_max.argtypes = [vp, i32, i64, vp, i64]
+    L.oracle_grandk_mn_quantize.argtypes = [vp, i64, vp, i64, vp, i32, u64, f32]
+    L.oracle_grandk_mn_dequant_accumulate.argtypes = [vp, i32, vp, i64, vp, i64, i32]
     L.oracle_ternary_words.argtypes = [i64]
     L.oracle_quantize_ternary.argtypes = [vp, vp, vp, i64, f32, f32]
     L.oracle_dequantize_ternary.argtypes = [vp, vp, i64]
@@ -218,6 +222,41 @@ def qsgd_mn_dequant_accumulate(comprs, n, b, L=None):
     comprs = [_c(c, np.uint32) for c in comprs]
     out = np.empty(n, np.float32)
     L.oracle_qsgd_mn_dequant_accumulate(_ptr_array(comprs), len(comprs), out.ctypes.data, n, b)
+    return out
+
+
+# ------------------------------------------------------------ GRandK-MN ----
+
+def grandk_mn_max(grads, index, L=None) -> np.float32:
+    """M = max |g_w[index[k]]| over workers and kept coordinates in [0, n)."""
+    L = L or lib()
+    grads = [_c(g, np.float32) for g in grads]
+    index = _c(index, np.int64)
+    n = grads[0].size
+    return np.float32(L.oracle_grandk_mn_max(_ptr_array(grads), len(grads), n,
+                                             index.ctypes.data, index.size))
+
+
+def grandk_mn_quantize(grad, index, b, seed, M, L=None):
+    """One worker's record of its kept coordinates (length K = index.size)."""
+    L = L or lib()
+    grad = _c(grad, np.float32)
+    index = _c(index, np.int64)
+    K = index.size
+    compr = np.zeros(int(L.oracle_qsgd_words(K, b)), np.uint32)
+    L.oracle_grandk_mn_quantize(grad.ctypes.data, grad.size, index.ctypes.data, K,
+                                compr.ctypes.data, b, seed, float(M))
+    return compr
+
+
+def grandk_mn_dequant_accumulate(comprs, index, n, b, L=None):
+    """The n-element merge: scaled level sums at the kept coordinates, +0 elsewhere."""
+    L = L or lib()
+    comprs = [_c(c, np.uint32) for c in comprs]
+    index = _c(index, np.int64)
+    out = np.full(n, np.nan, np.float32)     # an element left unwritten shows as NaN
+    L.oracle_grandk_mn_dequant_accumulate(_ptr_array(comprs), len(comprs), index.ctypes.data,
+                                          index.size, out.ctypes.data, n, b)
     return out
 
 

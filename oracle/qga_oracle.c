@@ -21,6 +21,9 @@
  *         compatible; it prints no formula.  The QSGD-MaxNorm steps below are
  *         this library's definition of the method (global max-norm scale,
  *         s = 2^(b-1)-1 levels, stochastic rounding, signed b-bit codes).
+ *         "Results" also names GlobalRandKMaxNorm compression (K = 10000) as
+ *         its sparsified variant, again without a formula; the GRandK-MN
+ *         functions state this library's reading of it.
  *   [SC11] J. Salmon, M. Moraes, R. Dror, D. Shaw, "Parallel Random Numbers:
  *         As Easy as 1, 2, 3", SC'11 -- the Philox4x32-10 generator.
  *
@@ -370,6 +373,77 @@ void oracle_qsgd_mn_dequant_accumulate(const uint32_t *const *compr, int W, floa
         for (int w = 0; w < W; ++w)
             sum += qsgd_level_at(compr[w], e, b);
         out[e] = (float)sum * step;
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* GlobalRandKMaxNorm (GRandK-MN): QSGD-MaxNorm of K shared coordinates */
+/* ------------------------------------------------------------------ */
+/* [GC] "Results" names GlobalRandKMaxNorm compression, with K = 10000, as the
+ * sparsified variant of QSGDMaxNorm and gives no formula.  This library's
+ * reading: every worker keeps the same K coordinates index[0..K-1] (drawn by
+ * the caller, shared by all workers, so the sparse vectors still add up in
+ * an all-reduce); the kept values x[k] = g[index[k]] form a K-vector that is
+ * quantized exactly as QSGD-MaxNorm quantizes a gradient (M = max |x| over
+ * all workers, draw k for position k, header [M, b, K]); the merge sums the
+ * levels, scales them once and scatters them back to their coordinates, every
+ * other coordinate of the n-element result being +0.  A coordinate outside
+ * [0, n) is skipped: it does not enter M, gets level 0 and is not stored. */
+
+static int index_in_range(int64_t i, int64_t n)
+{
+    return i >= 0 && i < n;
+}
+
+float oracle_grandk_mn_max(const float *const *grad, int W, int64_t n, const int64_t *index,
+                           int64_t K)
+{
+    float m = 0.0f;
+    for (int w = 0; w < W; ++w)
+        for (int64_t k = 0; k < K; ++k) {
+            if (!index_in_range(index[k], n))
+                continue;
+            float a = fabsf(grad[w][index[k]]);
+            if (a > m)
+                m = a;
+        }
+    return m;
+}
+
+void oracle_grandk_mn_quantize(const float *grad, int64_t n, const int64_t *index, int64_t K,
+                               uint32_t *compr, int b, uint64_t seed, float M)
+{
+    int per_word = 32 / b;
+    uint32_t mask = (1u << b) - 1u;
+    compr[0] = bits_of(M);
+    compr[1] = bits_of((float)b);
+    compr[2] = bits_of((float)K);
+    for (int64_t w = 0; w < (K * b + 31) / 32; ++w)
+        compr[3 + w] = 0u;
+    for (int64_t k = 0; k < K; ++k) {
+        int32_t q = 0;
+        if (index_in_range(index[k], n))
+            q = oracle_qsgd_level(grad[index[k]], M, b, seed, k);
+        uint32_t code = (uint32_t)q & mask;
+        compr[3 + k / per_word] |= code << (32 - b * (int)(k % per_word + 1));
+    }
+}
+
+void oracle_grandk_mn_dequant_accumulate(const uint32_t *const *compr, int W,
+                                         const int64_t *index, int64_t K, float *out, int64_t n,
+                                         int b)
+{
+    float M = float_of(compr[0][0]);
+    float step = M / (float)qsgd_levels(b);
+    for (int64_t e = 0; e < n; ++e)
+        out[e] = 0.0f;
+    for (int64_t k = 0; k < K; ++k) {
+        if (!index_in_range(index[k], n))
+            continue;
+        int32_t sum = 0;
+        for (int w = 0; w < W; ++w)
+            sum += qsgd_level_at(compr[w], k, b);
+        out[index[k]] = (float)sum * step;
     }
 }
 

@@ -578,4 +578,79 @@ def pin_ternary_dequantize_and_merge(L):
         assert Fraction(float(merged[e])) == total, e
 
 
+# ====================================================== GRandK-MN ====
+
+def _grandk_case(rng, n, K, W, sorted_index=False):
+    gs = [(rng.standard_normal(n) * 2).astype(np.float32) for _ in range(W)]
+    index = rng.choice(n, size=K, replace=False).astype(np.int64)
+    if sorted_index:
+        index.sort()
+    if K:
+        gs[W - 1][index[K // 2]] = -9.5          # the largest kept magnitude
+    return gs, index
+
+
+def pin_grandk_is_qsgd_of_kept_values(L):
+    """The kept coordinates' record is the (pinned) QSGD-MaxNorm record of the
+    K-vector g[index]: M is the library max over kept values of all workers,
+    draws follow the position in the index list, the header holds K; the
+    merge puts the QSGD merge of those records at the kept coordinates and
+    +0 everywhere else.  With index = 0..n-1 everything is plain QSGD-MN."""
+    rng = np.random.default_rng(41)
+    for b in (2, 4, 8):
+        for n, K, W in ((3001, 777, 3), (4099, 1, 2), (257, 257, 4), (1000, 33, 8)):
+            gs, index = _grandk_case(rng, n, K, W)
+            M = oracle.grandk_mn_max(gs, index, L)
+            kept = [g[index] for g in gs]
+            assert M == np.max(np.abs(np.stack(kept))) == oracle.qsgd_mn_max(kept, L)
+            recs = []
+            for w in range(W):
+                rec = oracle.grandk_mn_quantize(gs[w], index, b, 1234 + w, M, L)
+                assert np.array_equal(rec, oracle.qsgd_mn_quantize(kept[w], b, 1234 + w, M, L))
+                recs.append(rec)
+            out = oracle.grandk_mn_dequant_accumulate(recs, index, n, b, L)
+            want = np.zeros(n, np.float32)
+            want[index] = oracle.qsgd_mn_dequant_accumulate(recs, K, b, L)
+            assert np.array_equal(out.view(np.uint32), want.view(np.uint32)), (b, n, K)
+        # the identity selection is QSGD-MN itself
+        gs = [(rng.standard_normal(500) * 3).astype(np.float32) for _ in range(2)]
+        ident = np.arange(500, dtype=np.int64)
+        M = oracle.grandk_mn_max(gs, ident, L)
+        assert M == oracle.qsgd_mn_max(gs, L)
+        recs = [oracle.grandk_mn_quantize(g, ident, b, 9 + w, M, L) for w, g in enumerate(gs)]
+        assert all(np.array_equal(r, oracle.qsgd_mn_quantize(g, b, 9 + w, M, L))
+                   for w, (r, g) in enumerate(zip(recs, gs)))
+        assert np.array_equal(oracle.grandk_mn_dequant_accumulate(recs, ident, 500, b, L),
+                              oracle.qsgd_mn_dequant_accumulate(recs, 500, b, L))
+
+
+def pin_grandk_skips_outside_coordinates_and_empty(L):
+    """Coordinates outside [0, n) do not enter M, get level 0 and are not
+    stored; K = 0 gives a header-only record and an all +0 merge."""
+    rng = np.random.default_rng(43)
+    n = 600
+    for b in (2, 8):
+        gs, index = _grandk_case(rng, n, 40, 2)
+        index[[3, 17, 29]] = [-1, n, 1 << 40]
+        valid = (index >= 0) & (index < n)
+        M = oracle.grandk_mn_max(gs, index, L)
+        assert M == np.max(np.abs(np.stack([g[index[valid]] for g in gs])))
+        recs = []
+        for w, g in enumerate(gs):
+            x = np.zeros(index.size, np.float32)
+            x[valid] = g[index[valid]]
+            rec = oracle.grandk_mn_quantize(g, index, b, 70 + w, M, L)
+            assert np.array_equal(rec, oracle.qsgd_mn_quantize(x, b, 70 + w, M, L))
+            recs.append(rec)
+        out = oracle.grandk_mn_dequant_accumulate(recs, index, n, b, L)
+        want = np.zeros(n, np.float32)
+        want[index[valid]] = oracle.qsgd_mn_dequant_accumulate(recs, index.size, b, L)[valid]
+        assert np.array_equal(out.view(np.uint32), want.view(np.uint32))
+        empty = np.zeros(0, np.int64)
+        assert oracle.grandk_mn_max(gs, empty, L) == 0.0
+        rec0 = oracle.grandk_mn_quantize(gs[0], empty, b, 1, F32(2.0), L)
+        assert rec0.tolist() == [bits_of_f32(2.0), bits_of_f32(b), 0]
+        assert not oracle.grandk_mn_dequant_accumulate([rec0], empty, n, b, L).view(np.uint32).any()
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -68,12 +68,24 @@ MUTANTS = [
     ("qsgd lsb-first", "int shift = 32 - b * (int)(e % per_word + 1);\n        compr[3 + e / per_word] |=",
      "int shift = b * (int)(e % per_word);\n        compr[3 + e / per_word] |="),
     ("no sign extension", "        q -= (int32_t)(1u << b);", "        q += 0;"),
-    ("merge step 2^(b-1)", "float step = M / (float)qsgd_levels(b);",
-     "float step = M / (float)(1 << (b - 1));"),
+    ("merge step 2^(b-1)", "float step = M / (float)qsgd_levels(b);\n    for (int64_t e = 0; e < n; ++e) {",
+     "float step = M / (float)(1 << (b - 1));\n    for (int64_t e = 0; e < n; ++e) {"),
+    ("grandk merge step 2^(b-1)",
+     "float step = M / (float)qsgd_levels(b);\n    for (int64_t e = 0; e < n; ++e)\n",
+     "float step = M / (float)(1 << (b - 1));\n    for (int64_t e = 0; e < n; ++e)\n"),
     ("ternary base 4", "            value = value * 3 + trit;", "            value = value * 4 + trit;"),
     ("ternary least significant first", "    for (int64_t k = e % 5; k < 4; ++k)\n        value /= 3;",
      "    for (int64_t k = 0; k < e % 5; ++k)\n        value /= 3;"),
     ("ternary words per 16", "    return 3 + (n + 19) / 20;", "    return 3 + (n + 15) / 16;"),
+    ("grandk draw keyed on coordinate", "q = oracle_qsgd_level(grad[index[k]], M, b, seed, k);",
+     "q = oracle_qsgd_level(grad[index[k]], M, b, seed, index[k]);"),
+    ("grandk level of position k", "q = oracle_qsgd_level(grad[index[k]], M, b, seed, k);",
+     "q = oracle_qsgd_level(grad[k], M, b, seed, k);"),
+    ("grandk header holds n", "compr[2] = bits_of((float)K);", "compr[2] = bits_of((float)n);"),
+    ("grandk max over leading values", "float a = fabsf(grad[w][index[k]]);",
+     "float a = fabsf(grad[w][k]);"),
+    ("grandk merge not cleared", "    for (int64_t e = 0; e < n; ++e)\n        out[e] = 0.0f;\n", ""),
+    ("grandk scatter to position", "out[index[k]] = (float)sum * step;", "out[k] = (float)sum * step;"),
 ]
 
 

@@ -1,7 +1,8 @@
 """Seeded synthetic inputs for the tests and the benchmark.
 
 This module only draws numbers: gradients of the shapes and distributions of
-the five workloads below, residual initial values, outlier placement and the
+the five workloads below, residual initial values, outlier placement, the
+kept coordinates of the sparsified (GRandK) variant and the
 per-tensor thresholds of the bucket workload (a statistic of the drawn input,
 fixed before any quantization runs).  It holds none of the quantization
 arithmetic and imports neither the oracle nor the GPU library, so both sides
@@ -55,6 +56,12 @@ WORKLOADS = {
 QSGD_OUTLIER_MAGNITUDE = 50.0
 QSGD_OUTLIER_FRACTION = 0.001
 QSGD_SEED_BASE = 1234          # Philox seed of worker w is QSGD_SEED_BASE + w
+
+# GRandK-MaxNorm keeps K = 10000 coordinates (the value the gradient-compression
+# README's "Results" uses for every sparsified run) of the QSGD workload's
+# gradients; the shared index is drawn once from its own seed.
+GRANDK_K = 10_000
+GRANDK_INDEX_SEED = 4321
 
 
 def bert_base_shapes():
@@ -133,6 +140,13 @@ def qsgd_gradient(n: int, gen: torch.Generator, device):
         sign = torch.randint(0, 2, (k,), generator=gen, device=device).to(torch.float32) * 2 - 1
         x[idx] = sign * QSGD_OUTLIER_MAGNITUDE
     return x
+
+
+def grandk_index(n: int, K: int = GRANDK_K, seed: int = GRANDK_INDEX_SEED):
+    """K distinct coordinates of [0, n), uniform without replacement, in draw
+    order: the index every worker keeps (int64 numpy array)."""
+    import numpy as np
+    return np.random.default_rng(seed).choice(n, size=K, replace=False).astype(np.int64)
 
 
 def bert_bucket(w: Workload, worker: int, iteration: int, device="cpu", sizes=None):
