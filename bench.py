@@ -528,7 +528,36 @@ def time_rows(dev, stream, peak, reps=20, scale=1):
                                                           workload=f"8 records of {nq:,}, b={b}")
         del cq
 
-    del grads, out
+    # GRandK-MaxNorm: the same gradients, K = 10000 shared coordinates
+    K = workloads.GRANDK_K
+    index = torch.from_numpy(workloads.grandk_index(nq, K)).to(dev)
+    ip = vp(index.data_ptr())
+    t = _time_launches(stream, lambda: ok(L.qga_grandk_mn_max(gp, Wq, nq, ip, K, vp(M.data_ptr()), sp),
+                                          "grandk_max"), reps)
+    rows["grandk_mn_max_w8"] = _row(t, K * Wq, 4.0, peak, reps + 3, bound="latency",
+                                    workload=f"8 x {nq:,} fp32, K = {K:,} kept coordinates")
+    for b in wq.bits:
+        ck = [torch.empty(q.qga_qsgd_words(K, b), dtype=torch.int32, device=dev) for _ in range(Wq)]
+
+        def quant_k(k=0, b=b, ck=ck):
+            ok(L.qga_grandk_mn_quantize(vp(grads[k].data_ptr()), nq, ip, K, vp(ck[k].data_ptr()), b,
+                                        workloads.QSGD_SEED_BASE + k, vp(M.data_ptr()), sp),
+               "grandk_quantize")
+        for k in range(Wq):
+            quant_k(k)
+        t = _time_launches(stream, quant_k, reps)
+        rows[f"grandk_mn_quantize_b{b}"] = _row(t, K, 4 + 8 + b / 8, peak, reps + 3 + Wq,
+                                                bound="latency", workload=f"K = {K:,} of {nq:,}, b={b}")
+        carr = (ctypes.c_void_p * Wq)(*[cc.data_ptr() for cc in ck])
+        cp = ctypes.cast(carr, ctypes.POINTER(ctypes.c_void_p))
+        # the merge clears the n-element result (cudaMemsetAsync), then scatters K values
+        t = _time_launches(stream, lambda: ok(L.qga_grandk_mn_dequant_accumulate(
+            cp, Wq, ip, K, vp(out.data_ptr()), nq, b, sp), "grandk_merge"), reps)
+        rows[f"grandk_mn_dequant_accumulate_b{b}_w8"] = _row(
+            t, nq, 4 + (K * (8 + 4 + Wq * b / 8)) / nq, peak, reps + 3, bound="hbm (clear of out)",
+            workload=f"8 records of K = {K:,}, out of {nq:,}")
+        del ck
+    del grads, out, index
     torch.cuda.empty_cache()
     return rows
 

@@ -213,6 +213,40 @@ int qga_qsgd_mn_quantize(const float *grad, uint32_t *compr, int64_t n, int bits
 int qga_qsgd_mn_dequant_accumulate(const uint32_t *const *compr, int num_workers, float *out,
                                    int64_t n, int bits, cudaStream_t stream);
 
+/* ============================================ GRandK-MaxNorm, b bits ==
+ * GlobalRandKMaxNorm compression is named in [GC] "Results" (K = 10000) as
+ * the sparsified variant of QSGDMaxNorm, without a formula; this library
+ * defines it as follows.  All workers keep the same K coordinates index[k]
+ * (int64, drawn by the caller from a seed the workers share, distinct); the
+ * kept values x[k] = grad[index[k]] are quantized exactly as QSGD-MaxNorm
+ * quantizes a K-element gradient: M = max |x| over all workers, the draw u of
+ * position k (not of the coordinate), the record of qga_qsgd_words(K, bits)
+ * words with header [M, b, K].  The merge scatters the scaled level sums to
+ * their coordinates; every other coordinate of the result is +0.
+ * A coordinate outside [0, n) is skipped everywhere: it does not enter M, its
+ * level is 0 and nothing is stored for it.  With repeated coordinates the
+ * merge stores one of their values (which one is unspecified).
+ *   index  device int64[K], 8-byte aligned, owned by the caller; K >= 0. */
+
+/* M = max |grad_w[index[k]]| over w < num_workers and k < K, written to
+ * *max_out (device float, cleared first with cudaMemsetAsync); NaN skipped. */
+int qga_grandk_mn_max(const float *const *grad, int num_workers, int64_t n, const int64_t *index,
+                      int64_t k, float *max_out, cudaStream_t stream);
+
+/* One worker's record of its kept values; M read from *max_in (device).
+ *   grad   float[n];  compr uint32[qga_qsgd_words(k, bits)], overwritten
+ *   bits   2, 4 or 8 (others: QGA_ERR_UNSUPPORTED) */
+int qga_grandk_mn_quantize(const float *grad, int64_t n, const int64_t *index, int64_t k,
+                           uint32_t *compr, int bits, uint64_t seed, const float *max_in,
+                           cudaStream_t stream);
+
+/* Merge of W records over the same index: out (float[n]) is cleared to +0
+ * with cudaMemsetAsync, then out[index[k]] = (float)(sum_w q_w[k]) * (M / s),
+ * M from worker 0's header, M / s one binary32 division. */
+int qga_grandk_mn_dequant_accumulate(const uint32_t *const *compr, int num_workers,
+                                     const int64_t *index, int64_t k, float *out, int64_t n,
+                                     int bits, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

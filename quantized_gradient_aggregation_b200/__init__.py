@@ -11,8 +11,9 @@ quantized_gradient_aggregation_b200/build.py``).
 
 Methods: MXNet pull request #8342 "[WIP] 2bit gradient compression" (the 2-bit
 threshold quantizer with residual, its record format and the receiver-side
-merge) and the QSGD-MaxNorm b-bit scheme named in the gradient-compression
-README (vineeths96), as defined in ``include/qga.h``.
+merge) and the QSGD-MaxNorm b-bit scheme and its GlobalRandK sparsified
+variant named in the gradient-compression README (vineeths96), as defined in
+``include/qga.h``.
 """
 from __future__ import annotations
 
@@ -69,6 +70,9 @@ _SIGS = {
     "qga_qsgd_mn_max": (_i32, [_VPP, _i32, _i64, _vp, _vp]),
     "qga_qsgd_mn_quantize": (_i32, [_vp, _vp, _i64, _i32, _u64, _vp, _vp]),
     "qga_qsgd_mn_dequant_accumulate": (_i32, [_VPP, _i32, _vp, _i64, _i32, _vp]),
+    "qga_grandk_mn_max": (_i32, [_VPP, _i32, _i64, _vp, _i64, _vp, _vp]),
+    "qga_grandk_mn_quantize": (_i32, [_vp, _i64, _vp, _i64, _vp, _i32, _u64, _vp, _vp]),
+    "qga_grandk_mn_dequant_accumulate": (_i32, [_VPP, _i32, _vp, _i64, _vp, _i64, _i32, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -308,3 +312,44 @@ def qga_qsgd_mn_dequant_accumulate(comprs, out, bits, stream=None):
     _check(_lib.qga_qsgd_mn_dequant_accumulate(arr, len(comprs), _ptr(out), n, bits,
                                                _stream(stream, out.device)),
            "qga_qsgd_mn_dequant_accumulate")
+
+
+# ======================================================== GRandK-MN ====
+
+def qga_grandk_mn_max(grads, index, max_out, stream=None):
+    """M over the kept coordinates ``index`` (int64) of every worker's grad."""
+    n = grads[0].numel()
+    for i, g in enumerate(grads):
+        _need(g, torch.float32, n, f"grad[{i}]")
+    _need(index, torch.int64, None, "index")
+    _need(max_out, torch.float32, 1, "max_out")
+    arr, keep = _ptr_array(grads)
+    _check(_lib.qga_grandk_mn_max(arr, len(grads), n, _ptr(index), index.numel(), _ptr(max_out),
+                                  _stream(stream, max_out.device)),
+           "qga_grandk_mn_max")
+
+
+def qga_grandk_mn_quantize(grad, index, compr, bits, seed, max_in, stream=None):
+    _need(grad, torch.float32, None, "grad")
+    _need(index, torch.int64, None, "index")
+    _need(compr, torch.int32, qga_qsgd_words(index.numel(), bits), "compr")
+    _need(max_in, torch.float32, 1, "max_in")
+    _check(_lib.qga_grandk_mn_quantize(_ptr(grad), grad.numel(), _ptr(index), index.numel(),
+                                       _ptr(compr), bits, seed & ((1 << 64) - 1), _ptr(max_in),
+                                       _stream(stream, grad.device)),
+           "qga_grandk_mn_quantize")
+
+
+def qga_grandk_mn_dequant_accumulate(comprs, index, out, bits, stream=None):
+    """Merge into ``out`` (float32[n], overwritten): the scaled level sums at
+    the kept coordinates, +0 elsewhere."""
+    _need(out, torch.float32, None, "out")
+    _need(index, torch.int64, None, "index")
+    words = qga_qsgd_words(index.numel(), bits)
+    for i, c in enumerate(comprs):
+        _need(c, torch.int32, words, f"compr[{i}]")
+    arr, keep = _ptr_array(comprs)
+    _check(_lib.qga_grandk_mn_dequant_accumulate(arr, len(comprs), _ptr(index), index.numel(),
+                                                 _ptr(out), out.numel(), bits,
+                                                 _stream(stream, out.device)),
+           "qga_grandk_mn_dequant_accumulate")

@@ -38,7 +38,9 @@ def test_header_declares_the_boundary():
                  "qga_qsgd_words", "qga_qsgd_mn_max", "qga_qsgd_mn_quantize",
                  "qga_qsgd_mn_dequant_accumulate", "qga_strerror", "qga_last_cuda_error",
                  "qga_version", "qga_ternary_words", "qga_quantize_ternary",
-                 "qga_dequantize_ternary", "qga_dequant_accumulate_ternary"]:
+                 "qga_dequantize_ternary", "qga_dequant_accumulate_ternary",
+                 "qga_grandk_mn_max", "qga_grandk_mn_quantize",
+                 "qga_grandk_mn_dequant_accumulate"]:
         assert want in names, want
 
 
@@ -141,6 +143,25 @@ def test_invalid_arguments_are_rejected_before_any_cuda_call(qga):
     assert L.qga_qsgd_mn_dequant_accumulate(parr, 2, FAKE, 16, 5, None) == qga.QGA_ERR_UNSUPPORTED
     assert L.qga_qsgd_mn_dequant_accumulate(parr, 2, None, 16, 2, None) == E
     assert L.qga_qsgd_mn_dequant_accumulate(parr, 99, FAKE, 16, 2, None) == E
+    # GRandK-MN: index is int64 (8-byte aligned), K >= 0
+    assert L.qga_grandk_mn_max(parr, 2, 16, FAKE, -1, FAKE, None) == E
+    assert L.qga_grandk_mn_max(parr, 2, 16, None, 4, FAKE, None) == E
+    assert L.qga_grandk_mn_max(parr, 2, 16, FAKE + 4, 4, FAKE, None) == E
+    assert L.qga_grandk_mn_max(parr, 0, 16, FAKE, 4, FAKE, None) == E
+    assert L.qga_grandk_mn_max(ctypes.cast(bad, ctypes.POINTER(ctypes.c_void_p)), 2, 16, FAKE, 4,
+                               FAKE, None) == E
+    assert L.qga_grandk_mn_quantize(FAKE, 16, FAKE + 4, 4, FAKE, 2, 0, FAKE, None) == E
+    assert L.qga_grandk_mn_quantize(None, 16, FAKE, 4, FAKE, 2, 0, FAKE, None) == E
+    assert L.qga_grandk_mn_quantize(FAKE, 16, FAKE, 4, None, 2, 0, FAKE, None) == E
+    assert L.qga_grandk_mn_quantize(FAKE, 16, FAKE, 4, FAKE, 2, 0, None, None) == E
+    assert L.qga_grandk_mn_quantize(FAKE, -2, FAKE, 4, FAKE, 2, 0, FAKE, None) == E
+    assert L.qga_grandk_mn_quantize(FAKE, 16, FAKE, 4, FAKE, 6, 0, FAKE, None) == qga.QGA_ERR_UNSUPPORTED
+    assert L.qga_grandk_mn_dequant_accumulate(parr, 2, FAKE, 4, FAKE, 16, 3, None) == \
+        qga.QGA_ERR_UNSUPPORTED
+    assert L.qga_grandk_mn_dequant_accumulate(parr, 2, None, 4, FAKE, 16, 2, None) == E
+    assert L.qga_grandk_mn_dequant_accumulate(parr, 2, FAKE, 4, None, 16, 2, None) == E
+    assert L.qga_grandk_mn_dequant_accumulate(parr, 2, FAKE, -4, FAKE, 16, 2, None) == E
+    assert L.qga_grandk_mn_dequant_accumulate(parr, 65, FAKE, 4, FAKE, 16, 2, None) == E
     # dense ternary
     assert L.qga_ternary_words(-1) == E and L.qga_ternary_words(0) == 3 and L.qga_ternary_words(21) == 5
     assert L.qga_quantize_ternary(None, FAKE, FAKE, 16, -1.0, 1.0, None) == E
