@@ -130,17 +130,25 @@ __global__ void __launch_bounds__(kThreads)
                 gv[j] = make_float4(t[0], t[1], t[2], t[3]);
             }
         }
+        // the lane's four Philox chains side by side (independent, so their
+        // fixed-latency round dependencies overlap), then the levels
+        uint4 draws[kGroupsPerLane];
 #pragma unroll
         for (int j = 0; j < kGroupsPerLane; ++j) {
             const int64_t gi = g0 + j * kWarp + lane;
-            const uint4 r = philox4x32_10(
+            draws[j] = philox4x32_10(
                 make_uint4((uint32_t)gi, (uint32_t)((uint64_t)gi >> 32), 0u, 0u), key0, key1);
+        }
+#pragma unroll
+        for (int j = 0; j < kGroupsPerLane; ++j) {
+            const int64_t gi = g0 + j * kWarp + lane;
+            const uint4 r = draws[j];
             uint32_t c0, c1, c2, c3;
             if (fast) {
-                c0 = (uint32_t)qsgd_level<B>(gv[j].x, M, k, unit_draw(r.x)) & L::mask;
-                c1 = (uint32_t)qsgd_level<B>(gv[j].y, M, k, unit_draw(r.y)) & L::mask;
-                c2 = (uint32_t)qsgd_level<B>(gv[j].z, M, k, unit_draw(r.z)) & L::mask;
-                c3 = (uint32_t)qsgd_level<B>(gv[j].w, M, k, unit_draw(r.w)) & L::mask;
+                c0 = (uint32_t)qsgd_level<B>(gv[j].x, M, k, r.x) & L::mask;
+                c1 = (uint32_t)qsgd_level<B>(gv[j].y, M, k, r.y) & L::mask;
+                c2 = (uint32_t)qsgd_level<B>(gv[j].z, M, k, r.z) & L::mask;
+                c3 = (uint32_t)qsgd_level<B>(gv[j].w, M, k, r.w) & L::mask;
             } else {
                 c0 = (uint32_t)qsgd_level_exact<B>(gv[j].x, M, unit_draw(r.x)) & L::mask;
                 c1 = (uint32_t)qsgd_level_exact<B>(gv[j].y, M, unit_draw(r.y)) & L::mask;

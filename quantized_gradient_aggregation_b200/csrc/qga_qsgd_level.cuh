@@ -68,18 +68,22 @@ __device__ __forceinline__ int32_t qsgd_level_exact(float g, float M, float u)
 // 2^-14 away from an integer, floor(t') == floor(t); otherwise (or if t' is
 // not finite) the exact sequence decides.  Results are identical to
 // qsgd_level_exact for every input.
+//   x: the draw's output word; u = (x >> 8) 2^-24 enters the sum through one
+//   fused multiply-add, whose product is exact, so the sum is the same single
+//   rounding of |g| k + u as a separate add of u.
 template <int B>
-__device__ __forceinline__ int32_t qsgd_level(float g, float M, float k, float u)
+__device__ __forceinline__ int32_t qsgd_level(float g, float M, float k, uint32_t x)
 {
     constexpr float s = (float)Levels<B>::s;
     constexpr float kMargin = 0x1p-14f;
-    const float tf = __fadd_rn(__fmul_rn(fabsf(g), k), u);
+    const float m = __uint2float_rn(x >> 8); // exact: below 2^24
+    const float tf = __fmaf_rn(m, 0x1p-24f, __fmul_rn(fabsf(g), k));
     const float fl = floorf(tf);
     const float d = __fsub_rn(tf, fl); // exact
     // d in [2^-14, 1 - 2^-14], as one comparison (its rounding moves the
     // bound by at most 2^-25, far inside the slack of the margin)
     if (!(fabsf(__fsub_rn(d, 0.5f)) <= 0.5f - kMargin))
-        return qsgd_level_exact<B>(g, M, u);
+        return qsgd_level_exact<B>(g, M, __fmul_rn(m, 0x1p-24f));
     return (int32_t)copysignf(fminf(fl, s), g); // g = -0 gives 0
 }
 
