@@ -166,6 +166,16 @@ struct RecordSet {
     const uint32_t *rec[QGA_MAX_WORKERS];
 };
 
+// Of every QGA_TERNARY_TABLE_PERIOD consecutive workers, the first
+// QGA_TERNARY_TABLE_SHARE go through the pair table, the others through the
+// code masks.
+#ifndef QGA_TERNARY_TABLE_PERIOD
+#define QGA_TERNARY_TABLE_PERIOD 2
+#endif
+#ifndef QGA_TERNARY_TABLE_SHARE
+#define QGA_TERNARY_TABLE_SHARE 1
+#endif
+
 // kMerge: sum of W records from +0 in worker order (bit for bit the 2-bit
 // merge's sums); otherwise W == 1 and each element is its code's value.
 // As in the 2-bit merge, even workers go through a per-worker pair table
@@ -216,7 +226,7 @@ __global__ void __launch_bounds__(kThreads)
                 if (wb + i >= W) // warp-uniform
                     break;
                 const uint32_t word = words[i];
-                if (kMerge && (i & 1) == 0) {
+                if (kMerge && (i % QGA_TERNARY_TABLE_PERIOD) < QGA_TERNARY_TABLE_SHARE) {
                     // the 20 codes as a 40-bit string, element 0 in bits 39..38
                     const uint32_t c0 = s_codes[word & 0xFFu], c1 = s_codes[(word >> 8) & 0xFFu];
                     const uint32_t c2 = s_codes[(word >> 16) & 0xFFu], c3 = s_codes[word >> 24];
