@@ -94,7 +94,9 @@ def workload_config(w, n_gpus):
         "workload": (f"{w.name}: W={w.workers} simulated workers x n={w.n:,} fp32, "
                      f"g~Laplace(0,{w.scale:g}) (seeded synthetic, {w.iterations} iterations "
                      f"resident and cycled), residual carried, thresholds {w.neg_thr:g}/{w.pos_thr:g}; "
-                     "step = 8 quantize + 1 merge of 8 packed streams"),
+                     f"step = quantize of workers 1..{w.workers - 1}, then worker 0 (the reducing "
+                     f"worker) quantizes its own gradient and merges all {w.workers} records in one "
+                     "launch"),
         "n": w.n,
         "workers": w.workers,
         "l2": "every buffer (553 MB per gradient) is larger than the 126 MB L2; no flush",
@@ -290,10 +292,14 @@ def run_qga(args, rank, world, local_rank):
         if st:
             raise q.QGAError(st, "qga_quantize_2bit")
 
-    def merge():
-        st = L.qga_dequant_accumulate_2bit(cpp, W, ctypes.c_void_p(out.data_ptr()), n, sp)
+    def reduce(it):
+        # worker 0 is the reducing worker ([MX] Local kvstore): its own quantize
+        # and the merge of all W records are one launch
+        st = L.qga_quantize_merge_2bit(ctypes.c_void_p(grads[it][0].data_ptr()),
+                                       ctypes.c_void_p(res[0].data_ptr()), n, neg, pos, cpp, W, 0,
+                                       ctypes.c_void_p(out.data_ptr()), sp)
         if st:
-            raise q.QGAError(st, "qga_dequant_accumulate_2bit")
+            raise q.QGAError(st, "qga_quantize_merge_2bit")
 
     def barrier():
         if world > 1:
@@ -302,29 +308,29 @@ def run_qga(args, rank, world, local_rank):
     sampler = ClockSampler(gpu_id_for(local_rank))
     time.sleep(0.3)
     for s in range(args.warmup):
-        for k in range(W):
+        for k in range(1, W):
             quant(s % iters, k)
-        merge()
+        reduce(s % iters)
     torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
 
     K = args.steps
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
-    q_ev = [(ev(), ev()) for _ in range(K * W)]
+    q_ev = [(ev(), ev()) for _ in range(K * (W - 1))]
     m_ev = [(ev(), ev()) for _ in range(K)]
     start, end = ev(), ev()
     start.record(stream)
     for s in range(K):
         it = (args.warmup + s) % iters
-        for k in range(W):
-            a, b = q_ev[s * W + k]
+        for k in range(1, W):
+            a, b = q_ev[s * (W - 1) + k - 1]
             a.record(stream)
             quant(it, k)
             b.record(stream)
         a, b = m_ev[s]
         a.record(stream)
-        merge()
+        reduce(it)
         b.record(stream)
     end.record(stream)
     torch.cuda.synchronize()
@@ -337,7 +343,7 @@ def run_qga(args, rank, world, local_rank):
     merge_ms = statistics.fmean(a.elapsed_time(b) for a, b in m_ev)
     total_ms, quant_ms, merge_ms = max_over_ranks([total_ms, quant_ms, merge_ms], world, dev)
 
-    e2e = None if args.no_e2e else run_e2e(args, w, grads[0], res, comprs, out, quant, merge,
+    e2e = None if args.no_e2e else run_e2e(args, w, grads[0], res, comprs, out, quant, reduce,
                                            stream, world, dev)
     del grads, res, comprs, out
     torch.cuda.empty_cache()
@@ -348,7 +354,7 @@ def run_qga(args, rank, world, local_rank):
         return
     peak, peak_kind = measured_peaks()
     quant_gbs = QUANT_BYTES_PER_ELEM * n / (quant_ms * 1e-3) / 1e9
-    merge_gbs = (0.25 * W + 4) * n / (merge_ms * 1e-3) / 1e9
+    merge_gbs = (QUANT_BYTES_PER_ELEM + 0.25 * (W - 1) + 4) * n / (merge_ms * 1e-3) / 1e9
     traffic_per_elem = MEASURED_TRAFFIC.get(csrc_hash(QUANT_SOURCES))
     line = {
         "metric": METRIC,
@@ -369,12 +375,13 @@ def run_qga(args, rank, world, local_rank):
             "quantize_2bit": {"us": quant_ms * 1e3, "gelem_s": n / (quant_ms * 1e-3) / 1e9,
                               "gb_s": quant_gbs, "frac_of_peak": quant_gbs / peak,
                               "frac_of_8TBs": quant_gbs / 8000.0},
-            "dequant_accumulate_2bit_w8": {"us": merge_ms * 1e3,
-                                           "gelem_s": n / (merge_ms * 1e-3) / 1e9,
-                                           "gb_s": merge_gbs, "frac_of_peak": merge_gbs / peak,
-                                           "frac_of_8TBs": merge_gbs / 8000.0},
+            "quantize_merge_2bit_w8": {"us": merge_ms * 1e3,
+                                       "gelem_s": n / (merge_ms * 1e-3) / 1e9,
+                                       "gb_s": merge_gbs, "frac_of_peak": merge_gbs / peak,
+                                       "frac_of_8TBs": merge_gbs / 8000.0,
+                                       "bytes_per_elem": QUANT_BYTES_PER_ELEM + 0.25 * (W - 1) + 4},
         },
-        "gpu_launches": K * (W + 1),
+        "gpu_launches": K * W,
         "clocks": clocks,
         "csrc": csrc_hash(),
         "quantize_sources": csrc_hash(QUANT_SOURCES),
@@ -442,7 +449,24 @@ def time_rows(dev, stream, peak, reps=20, scale=1):
     t = _time_launches(stream, lambda: ok(L.qga_dequantize_2bit(vp(c.data_ptr()), vp(out.data_ptr()),
                                                                 n, sp), "dequantize"), reps)
     rows["dequantize_2bit"] = _row(t, n, 4.25, peak, reps + 3, workload=f"vgg16 record, n={n:,}")
-    del c
+
+    # the reducing worker's fused step: quantize worker 0, merge 8 records
+    others = [c.clone() for _ in range(w.workers - 1)]
+    c_own = torch.empty_like(c)
+    rarr = (ctypes.c_void_p * w.workers)(*[x.data_ptr() for x in [c_own] + others])
+    rp = ctypes.cast(rarr, ctypes.POINTER(ctypes.c_void_p))
+    t = _time_launches(stream, lambda: ok(L.qga_quantize_merge_2bit(
+        vp(g.data_ptr()), vp(r.data_ptr()), n, w.neg_thr, w.pos_thr, rp, w.workers, 0,
+        vp(out.data_ptr()), sp), "quantize_merge"), reps)
+    rows["quantize_merge_2bit_w8_alone"] = _row(t, n, 12.25 + 0.25 * (w.workers - 1) + 4, peak,
+                                                reps + 3,
+                                                workload=f"vgg16 worker 0 + 7 received records, n={n:,}")
+    # the merge alone (A8): 8 records
+    t = _time_launches(stream, lambda: ok(L.qga_dequant_accumulate_2bit(
+        rp, w.workers, vp(out.data_ptr()), n, sp), "merge"), reps)
+    rows["dequant_accumulate_2bit_w8"] = _row(t, n, 0.25 * w.workers + 4, peak, reps + 3,
+                                              workload=f"8 records of n={n:,}")
+    del c, others, c_own
 
     # dense ternary records (5 codes per byte): quantize and the 8-worker merge
     ct = [torch.empty(q.qga_ternary_words(n), dtype=torch.int32, device=dev) for _ in range(w.workers)]
@@ -562,12 +586,14 @@ def time_rows(dev, stream, peak, reps=20, scale=1):
     return rows
 
 
-def run_e2e(args, w, dev_grads, res, comprs, out, quant, merge, stream, world, dev):
+def run_e2e(args, w, dev_grads, res, comprs, out, quant, reduce, stream, world, dev):
     """Same step with the gradients arriving from pinned host memory and the
     aggregate read back, copies inside the timed region.  Copies run on a
-    second stream: worker k's upload overlaps the quantize of worker k - 1,
-    and the aggregate's download (the other PCIe direction) overlaps the
-    next step's uploads; events order every reuse of a buffer."""
+    second stream: worker k's upload overlaps the quantize of the worker
+    before it, and the aggregate's download (the other PCIe direction)
+    overlaps the next step's uploads; events order every reuse of a buffer.
+    Worker 0, the reducing worker, comes last: its quantize and the merge
+    are one launch."""
     import torch
     n, W = w.n, w.workers
     host = [torch.empty(n, dtype=torch.float32, pin_memory=True) for _ in range(W)]
@@ -585,17 +611,19 @@ def run_e2e(args, w, dev_grads, res, comprs, out, quant, merge, stream, world, d
     downloaded.record(stream)
 
     def step():
-        for k in range(W):
+        for k in list(range(1, W)) + [0]:
             with torch.cuda.stream(copy_stream):
                 copy_stream.wait_event(consumed[k])      # previous quantize of worker k is done
                 dev_grads[k].copy_(host[k], non_blocking=True)
                 landed[k].record(copy_stream)
             stream.wait_event(landed[k])
-            quant(0, k)
+            if k:
+                quant(0, k)
+            else:
+                stream.wait_event(downloaded)            # previous aggregate has left the device
+                reduce(0)
+                merged.record(stream)
             consumed[k].record(stream)
-        stream.wait_event(downloaded)                    # previous aggregate has left the device
-        merge()
-        merged.record(stream)
         with torch.cuda.stream(copy_stream):
             copy_stream.wait_event(merged)
             host_out.copy_(out, non_blocking=True)
@@ -618,8 +646,8 @@ def run_e2e(args, w, dev_grads, res, comprs, out, quant, merge, stream, world, d
     (ms,) = max_over_ranks([a.elapsed_time(b)], world, dev)
     return {"value": job_gelem_per_s(world, W, n, K, ms), "unit": "Gelem/s",
             "h2d_bytes_per_step": W * n * 4, "d2h_bytes_per_step": n * 4, "steps": K,
-            "path": "pinned host gradients -> cudaMemcpyAsync (copy stream) -> qga_quantize_2bit x8 "
-                    "-> qga_dequant_accumulate_2bit -> pinned host aggregate (copy stream)"}
+            "path": "pinned host gradients -> cudaMemcpyAsync (copy stream) -> qga_quantize_2bit x7 "
+                    "-> qga_quantize_merge_2bit (worker 0) -> pinned host aggregate (copy stream)"}
 
 
 def main():

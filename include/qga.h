@@ -116,6 +116,25 @@ int qga_dequantize_2bit(const uint32_t *compr, float *out, int64_t n, cudaStream
 int qga_dequant_accumulate_2bit(const uint32_t *const *compr, int num_workers, float *out,
                                 int64_t n, cudaStream_t stream);
 
+/* The reducing worker's step of [MX] "Local kvstore" in one launch: the
+ * device that merges the workers' gradients also quantizes its own ([MX]
+ * "Questions", 1).  Worker `own`'s gradient is quantized exactly as by
+ * qga_quantize_2bit (residual updated in place, record written to
+ * compr[own]), and the W records are merged exactly as by
+ * qga_dequant_accumulate_2bit (worker order 0..W-1, own included).  The
+ * results are bit for bit those of the two calls in sequence.
+ *   grad, residual  float[n] of worker `own`
+ *   compr           HOST array of W device pointers to records of n
+ *                   elements; compr[own] is overwritten, the others are read
+ *   own             0 .. W-1;  num_workers 1 .. QGA_MAX_WORKERS
+ *   out             float[n], overwritten; no buffer may overlap another.
+ * 32-byte-aligned grad and residual with a 16-byte-aligned out take the
+ * vector path, other element-aligned pointers a scalar path with identical
+ * results. */
+int qga_quantize_merge_2bit(const float *grad, float *residual, int64_t n, float neg_threshold,
+                            float pos_threshold, uint32_t *const *compr, int num_workers, int own,
+                            float *out, cudaStream_t stream);
+
 /* ---------------------------------------------------------- 2-bit bucket --
  * A bucket is T tensors quantized in ONE launch.  Its compressed form is the
  * T standalone records one after the other (tensor t's record starts at word

@@ -66,6 +66,7 @@ _SIGS = {
     "qga_quantize_ternary": (_i32, [_vp, _vp, _vp, _i64, _f32, _f32, _vp]),
     "qga_dequantize_ternary": (_i32, [_vp, _vp, _i64, _vp]),
     "qga_dequant_accumulate_ternary": (_i32, [_VPP, _i32, _vp, _i64, _vp]),
+    "qga_quantize_merge_2bit": (_i32, [_vp, _vp, _i64, _f32, _f32, _VPP, _i32, _i32, _vp, _vp]),
     "qga_qsgd_words": (_i64, [_i64, _i32]),
     "qga_qsgd_mn_max": (_i32, [_VPP, _i32, _i64, _vp, _vp]),
     "qga_qsgd_mn_quantize": (_i32, [_vp, _vp, _i64, _i32, _u64, _vp, _vp]),
@@ -181,6 +182,24 @@ def qga_dequant_accumulate_2bit(comprs, out, stream=None):
     _check(_lib.qga_dequant_accumulate_2bit(arr, len(comprs), _ptr(out), n,
                                             _stream(stream, out.device)),
            "qga_dequant_accumulate_2bit")
+
+
+def qga_quantize_merge_2bit(grad, residual, comprs, own, neg_threshold, pos_threshold, out,
+                            stream=None):
+    """The reducing worker's step: quantize worker ``own``'s gradient into
+    ``comprs[own]`` and merge all records into ``out``, in one launch."""
+    n = residual.numel()
+    _need(grad, torch.float32, n, "grad")
+    _need(residual, torch.float32, None, "residual")
+    _need(out, torch.float32, n, "out")
+    words = qga_2bit_words(n)
+    for i, c in enumerate(comprs):
+        _need(c, torch.int32, words, f"compr[{i}]")
+    arr, keep = _ptr_array(comprs)
+    _check(_lib.qga_quantize_merge_2bit(_ptr(grad), _ptr(residual), n, float(neg_threshold),
+                                        float(pos_threshold), arr, len(comprs), int(own), _ptr(out),
+                                        _stream(stream, residual.device)),
+           "qga_quantize_merge_2bit")
 
 
 def qga_2bit_bucket_words(sizes) -> int:

@@ -40,7 +40,7 @@ def test_header_declares_the_boundary():
                  "qga_version", "qga_ternary_words", "qga_quantize_ternary",
                  "qga_dequantize_ternary", "qga_dequant_accumulate_ternary",
                  "qga_grandk_mn_max", "qga_grandk_mn_quantize",
-                 "qga_grandk_mn_dequant_accumulate"]:
+                 "qga_grandk_mn_dequant_accumulate", "qga_quantize_merge_2bit"]:
         assert want in names, want
 
 
@@ -119,6 +119,18 @@ def test_invalid_arguments_are_rejected_before_any_cuda_call(qga):
     bad = (ctypes.c_void_p * 2)(FAKE, 0)
     assert L.qga_dequant_accumulate_2bit(ctypes.cast(bad, ctypes.POINTER(ctypes.c_void_p)), 2,
                                          FAKE, 16, None) == E
+    # quantize + merge of the reducing worker
+    assert L.qga_quantize_merge_2bit(FAKE, FAKE, 16, -1.0, 1.0, parr, 2, 2, FAKE, None) == E
+    assert L.qga_quantize_merge_2bit(FAKE, FAKE, 16, -1.0, 1.0, parr, 2, -1, FAKE, None) == E
+    assert L.qga_quantize_merge_2bit(FAKE, FAKE, 16, nan, 1.0, parr, 2, 0, FAKE, None) == E
+    assert L.qga_quantize_merge_2bit(FAKE, FAKE, -1, -1.0, 1.0, parr, 2, 0, FAKE, None) == E
+    assert L.qga_quantize_merge_2bit(None, FAKE, 16, -1.0, 1.0, parr, 2, 0, FAKE, None) == E
+    assert L.qga_quantize_merge_2bit(FAKE, FAKE, 16, -1.0, 1.0, parr, 2, 0, None, None) == E
+    assert L.qga_quantize_merge_2bit(FAKE, FAKE + 2, 16, -1.0, 1.0, parr, 2, 0, FAKE, None) == E
+    assert L.qga_quantize_merge_2bit(FAKE, FAKE, 16, -1.0, 1.0, parr, 0, 0, FAKE, None) == E
+    assert L.qga_quantize_merge_2bit(FAKE, FAKE, 16, -1.0, 1.0,
+                                     ctypes.cast(bad, ctypes.POINTER(ctypes.c_void_p)), 2, 0, FAKE,
+                                     None) == E
     # bucket
     T = qga.qga_bucket_tensor
     rows = (T * 2)(T(FAKE, FAKE, 16, -1.0, 1.0), T(FAKE, FAKE, -1, -1.0, 1.0))
