@@ -60,6 +60,43 @@ def test_two_bit_step_in_a_cuda_graph():
     assert np.array_equal(_bits([out_g])[0], _bits([out_e])[0])
 
 
+def test_reducing_worker_step_in_a_cuda_graph():
+    """The bench's step shape: quantizes of workers 1..W-1, then worker 0's
+    fused quantize + merge; captured once, replayed, equal to eager calls."""
+    q = qga()
+    n, W = 200_003, 4
+    gen = torch.Generator(device=DEV)
+    gen.manual_seed(10)
+    grads = [torch.randn(n, device=DEV, generator=gen) for _ in range(W)]
+    res0 = [torch.rand(n, device=DEV, generator=gen) - 0.5 for _ in range(W)]
+
+    def step(res, comprs, out):
+        for k in range(1, W):
+            q.qga_quantize_2bit(grads[k], res[k], comprs[k], -0.5, 0.5)
+        q.qga_quantize_merge_2bit(grads[0], res[0], comprs, 0, -0.5, 0.5, out)
+
+    res_e = [r.clone() for r in res0]
+    comprs_e = [torch.empty(q.qga_2bit_words(n), dtype=torch.int32, device=DEV) for _ in range(W)]
+    out_e = torch.empty(n, device=DEV)
+    for _ in range(2):
+        step(res_e, comprs_e, out_e)
+    res_g = [r.clone() for r in res0]
+    comprs_g = [torch.empty_like(c) for c in comprs_e]
+    out_g = torch.empty(n, device=DEV)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side):
+            step(res_g, comprs_g, out_g)
+    for _ in range(2):
+        graph.replay()
+    torch.cuda.synchronize()
+    assert all(np.array_equal(a, b) for a, b in zip(_bits(res_g), _bits(res_e)))
+    assert all(np.array_equal(a, b) for a, b in zip(_bits(comprs_g), _bits(comprs_e)))
+    assert np.array_equal(_bits([out_g])[0], _bits([out_e])[0])
+
+
 def test_bucket_and_qsgd_in_a_cuda_graph():
     q = qga()
     gen = torch.Generator(device=DEV)
