@@ -182,11 +182,14 @@ struct RecordSet {
 // (shared loads + paired adds) and odd workers through code masks and
 // predicated adds (skipping the exact +0 adds of code 00), so that neither
 // the integer pipe nor the load/store pipe saturates alone.
-template <bool kVec, bool kMerge>
+// kW > 0: compiled for exactly kW workers (record pointers from the kernel
+// parameters and loop bounds are constants); kW == 0: any W.
+template <bool kVec, bool kMerge, int kW>
 __global__ void __launch_bounds__(kThreads)
-    decode_ternary_kernel(const __grid_constant__ RecordSet set, int W, float *__restrict__ out,
-                          int64_t n)
+    decode_ternary_kernel(const __grid_constant__ RecordSet set, int W_runtime,
+                          float *__restrict__ out, int64_t n)
 {
+    const int W = kW > 0 ? kW : W_runtime;
     __shared__ uint16_t s_masks[256], s_codes[256];
     __shared__ const uint32_t *s_payload[QGA_MAX_WORKERS];
     __shared__ float s_neg[QGA_MAX_WORKERS], s_pos[QGA_MAX_WORKERS];
@@ -220,7 +223,9 @@ __global__ void __launch_bounds__(kThreads)
             uint32_t words[kBatch];
 #pragma unroll
             for (int i = 0; i < kBatch; ++i)
-                words[i] = (ok && wb + i < W) ? ld_stream_u32(s_payload[wb + i] + w) : 0u;
+                words[i] = (ok && wb + i < W)
+                               ? ld_stream_u32((kW > 0 ? set.rec[wb + i] + 3 : s_payload[wb + i]) + w)
+                               : 0u;
 #pragma unroll
             for (int i = 0; i < kBatch; ++i) {
                 if (wb + i >= W) // warp-uniform
@@ -275,34 +280,52 @@ __global__ void __launch_bounds__(kThreads)
     }
 }
 
-std::atomic<int> occ_tq[2][64], occ_td[2][2][64];
+std::atomic<int> occ_tq[2][64], occ_td[2][2][9][64]; // td: [vec][merge][kW]
 
 unsigned warps_grid(int64_t warp_items, int resident)
 {
     return grid_for((warp_items + kWarpsPerBlock - 1) / kWarpsPerBlock, resident);
 }
 
+template <bool kVec, bool kMerge, int kW>
+void launch_decode_k(const RecordSet &set, int W, float *out, int64_t n, cudaStream_t stream)
+{
+    const int64_t tiles = ((n + 19) / 20 + kWarp - 1) / kWarp;
+    auto k = decode_ternary_kernel<kVec, kMerge, kW>;
+    k<<<warps_grid(tiles, resident_blocks(k, kThreads, occ_td[kVec][kMerge][kW])), kThreads, 0,
+        stream>>>(set, W, out, n);
+}
+
+template <bool kVec>
+void launch_merge_v(const RecordSet &set, int W, float *out, int64_t n, cudaStream_t stream)
+{
+    switch (W) {
+    case 1: launch_decode_k<kVec, true, 1>(set, W, out, n, stream); break;
+    case 2: launch_decode_k<kVec, true, 2>(set, W, out, n, stream); break;
+    case 3: launch_decode_k<kVec, true, 3>(set, W, out, n, stream); break;
+    case 4: launch_decode_k<kVec, true, 4>(set, W, out, n, stream); break;
+    case 5: launch_decode_k<kVec, true, 5>(set, W, out, n, stream); break;
+    case 6: launch_decode_k<kVec, true, 6>(set, W, out, n, stream); break;
+    case 7: launch_decode_k<kVec, true, 7>(set, W, out, n, stream); break;
+    case 8: launch_decode_k<kVec, true, 8>(set, W, out, n, stream); break;
+    default: launch_decode_k<kVec, true, 0>(set, W, out, n, stream); break;
+    }
+}
+
 int launch_decode(const RecordSet &set, int W, float *out, int64_t n, cudaStream_t stream,
                   bool merge)
 {
-    const int64_t tiles = ((n + 19) / 20 + kWarp - 1) / kWarp;
     const bool vec = aligned(out, 16);
     if (merge) {
-        if (vec) {
-            auto k = decode_ternary_kernel<true, true>;
-            k<<<warps_grid(tiles, resident_blocks(k, kThreads, occ_td[1][1])), kThreads, 0, stream>>>(set, W, out, n);
-        } else {
-            auto k = decode_ternary_kernel<false, true>;
-            k<<<warps_grid(tiles, resident_blocks(k, kThreads, occ_td[0][1])), kThreads, 0, stream>>>(set, W, out, n);
-        }
+        if (vec)
+            launch_merge_v<true>(set, W, out, n, stream);
+        else
+            launch_merge_v<false>(set, W, out, n, stream);
     } else {
-        if (vec) {
-            auto k = decode_ternary_kernel<true, false>;
-            k<<<warps_grid(tiles, resident_blocks(k, kThreads, occ_td[1][0])), kThreads, 0, stream>>>(set, W, out, n);
-        } else {
-            auto k = decode_ternary_kernel<false, false>;
-            k<<<warps_grid(tiles, resident_blocks(k, kThreads, occ_td[0][0])), kThreads, 0, stream>>>(set, W, out, n);
-        }
+        if (vec)
+            launch_decode_k<true, false, 1>(set, 1, out, n, stream);
+        else
+            launch_decode_k<false, false, 1>(set, 1, out, n, stream);
     }
     return launch_status();
 }
