@@ -34,7 +34,9 @@ constexpr int kWarpsPerBlock = kThreads / kWarp;
 // Blocks per SM the register budget is fitted to (64 registers a thread at 4).
 // Measured at n = 138M, W = 8: 4 blocks 426 us, 3 blocks 428 us, 2 blocks
 // 496 us.  Issuing both words' loads before either is quantized (470-618 us)
-// and prefetching the next slice into L2 (570-602 us) were slower.
+// and prefetching the next slice into L2 (570-602 us) were slower; issuing
+// the received records' loads before the own quantize changed nothing
+// (426 us, at 3 blocks to avoid spills).
 #ifndef QGA_LOCAL_REDUCE_MIN_BLOCKS
 #define QGA_LOCAL_REDUCE_MIN_BLOCKS 4
 #endif
