@@ -101,17 +101,24 @@ std::atomic<int> occ_q_f32_v[64], occ_q_f32_s[64], occ_q_bf16_v[64], occ_q_bf16_
 std::atomic<int> occ_dq_v[64], occ_dq_s[64];
 std::atomic<int> occ_acc[2][9][64]; // [vec][kW][device]
 
-unsigned tiles_grid(int64_t n, int resident, int64_t elems_per_warp = kTileElems)
+// Grid waves (see grid_for), measured at n = 138M: quantize 1 / 8 / 16 / 32 /
+// 128 waves 270-286 / 263 / 259 / 256 / 258 us; dequantize 109 / 97 / 96 /
+// 101 us at 1 / 8 / 16 / 32; merge (W = 8) 180 / 174 / 176 / 181 us at
+// 1 / 8 / 16 / 32.
+constexpr int kQuantizeWaves = 32, kDequantizeWaves = 16, kMergeWaves = 8;
+
+unsigned tiles_grid(int64_t n, int resident, int64_t elems_per_warp, int waves)
 {
     const int64_t tiles = (n + elems_per_warp - 1) / elems_per_warp;
-    return grid_for((tiles + kWarpsPerBlock - 1) / kWarpsPerBlock, resident);
+    return grid_for((tiles + kWarpsPerBlock - 1) / kWarpsPerBlock, resident, waves);
 }
 
 template <bool kVec, int kW>
 void launch_merge_k(const RecordSet &set, int W, float *out, int64_t n, cudaStream_t stream)
 {
     auto k = dequant_accumulate_2bit_kernel<kVec, kW>;
-    k<<<tiles_grid(n, resident_blocks(k, kThreads, occ_acc[kVec][kW]), kSliceElems), kThreads, 0,
+    k<<<tiles_grid(n, resident_blocks(k, kThreads, occ_acc[kVec][kW]), kSliceElems, kMergeWaves),
+        kThreads, 0,
         stream>>>(set, W, out, n);
 }
 
@@ -152,11 +159,13 @@ int launch_quantize(const G *grad, float *residual, uint32_t *compr, int64_t n, 
     constexpr int64_t kElems = quantize_tile_elems<G>();
     if (vec) {
         auto k = quantize_2bit_kernel<G, true>;
-        k<<<tiles_grid(n, resident_blocks(k, kThreads, occ_v), kElems), kThreads, 0, stream>>>(
+        k<<<tiles_grid(n, resident_blocks(k, kThreads, occ_v), kElems, kQuantizeWaves), kThreads, 0,
+            stream>>>(
             grad, residual, compr, n, neg, pos);
     } else {
         auto k = quantize_2bit_kernel<G, false>;
-        k<<<tiles_grid(n, resident_blocks(k, kThreads, occ_s), kElems), kThreads, 0, stream>>>(
+        k<<<tiles_grid(n, resident_blocks(k, kThreads, occ_s), kElems, kQuantizeWaves), kThreads, 0,
+            stream>>>(
             grad, residual, compr, n, neg, pos);
     }
     return launch_status();
@@ -200,10 +209,12 @@ extern "C" int qga_dequantize_2bit(const uint32_t *compr, float *out, int64_t n,
         return QGA_ERR_INVALID_ARG;
     if (aligned(out, 16)) {
         auto k = dequantize_2bit_kernel<true>;
-        k<<<tiles_grid(n, resident_blocks(k, kThreads, occ_dq_v)), kThreads, 0, stream>>>(compr, out, n);
+        k<<<tiles_grid(n, resident_blocks(k, kThreads, occ_dq_v), kTileElems, kDequantizeWaves),
+            kThreads, 0, stream>>>(compr, out, n);
     } else {
         auto k = dequantize_2bit_kernel<false>;
-        k<<<tiles_grid(n, resident_blocks(k, kThreads, occ_dq_s)), kThreads, 0, stream>>>(compr, out, n);
+        k<<<tiles_grid(n, resident_blocks(k, kThreads, occ_dq_s), kTileElems, kDequantizeWaves),
+            kThreads, 0, stream>>>(compr, out, n);
     }
     return launch_status();
 }

@@ -311,19 +311,27 @@ std::atomic<int> occ_m[3][2][64];
 
 int bits_slot(int bits) { return bits == 2 ? 0 : (bits == 4 ? 1 : (bits == 8 ? 2 : -1)); }
 
+// Grid waves (see grid_for), measured at n = 2^27: quantize b = 2 / 4 / 8
+// 220 / 218 / 197 us at 1 wave, 205 / 203 / 185 at 8, 205 / 203 / 187 at 16;
+// merge (W = 8) b = 2 150 / 148 / 148, b = 4 231 / 206 / 201, b = 8 263 / 268 /
+// 266 us at 1 / 8 / 16 waves.  The max stays persistent (one atomic per block;
+// 606 / 602 / 606 / 696 us at 1 / 8 / 16 / 32).
+constexpr int kQsgdQuantizeWaves = 8;
+template <int B> constexpr int kQsgdMergeWaves = B == 8 ? 1 : 16;
+
 template <int B>
 unsigned merge_grid(int64_t n, int resident)
 {
     const int64_t nwords = (n * B + 31) >> 5;
     const int64_t per_block = (int64_t)kThreads * Swar<B>::kSlots;
-    return grid_for((nwords + per_block - 1) / per_block, resident);
+    return grid_for((nwords + per_block - 1) / per_block, resident, kQsgdMergeWaves<B>);
 }
 
 unsigned group_grid(int64_t n, int resident)
 {
     const int64_t groups = (n + 3) >> 2;
     const int64_t tiles = (groups + kTileGroups - 1) / kTileGroups;
-    return grid_for((tiles + kWarpsPerBlock - 1) / kWarpsPerBlock, resident);
+    return grid_for((tiles + kWarpsPerBlock - 1) / kWarpsPerBlock, resident, kQsgdQuantizeWaves);
 }
 
 template <int B>

@@ -282,9 +282,14 @@ __global__ void __launch_bounds__(kThreads)
 
 std::atomic<int> occ_tq[2][64], occ_td[2][2][9][64]; // td: [vec][merge][kW]
 
-unsigned warps_grid(int64_t warp_items, int resident)
+// Grid waves (see grid_for), measured at n = 138M: quantize 287 / 253 / 247 /
+// 243 / 240 us at 1 / 8 / 16 / 32 / 128 waves; merge (W = 8) 206 / 199 / 206
+// / 224 us at 1 / 8 / 16 / 32.
+constexpr int kTernaryQuantizeWaves = 32, kTernaryDecodeWaves = 8;
+
+unsigned warps_grid(int64_t warp_items, int resident, int waves)
 {
-    return grid_for((warp_items + kWarpsPerBlock - 1) / kWarpsPerBlock, resident);
+    return grid_for((warp_items + kWarpsPerBlock - 1) / kWarpsPerBlock, resident, waves);
 }
 
 template <bool kVec, bool kMerge, int kW>
@@ -292,7 +297,8 @@ void launch_decode_k(const RecordSet &set, int W, float *out, int64_t n, cudaStr
 {
     const int64_t tiles = ((n + 19) / 20 + kWarp - 1) / kWarp;
     auto k = decode_ternary_kernel<kVec, kMerge, kW>;
-    k<<<warps_grid(tiles, resident_blocks(k, kThreads, occ_td[kVec][kMerge][kW])), kThreads, 0,
+    k<<<warps_grid(tiles, resident_blocks(k, kThreads, occ_td[kVec][kMerge][kW]), kTernaryDecodeWaves),
+        kThreads, 0,
         stream>>>(set, W, out, n);
 }
 
@@ -353,11 +359,13 @@ extern "C" int qga_quantize_ternary(const float *grad, float *residual, uint32_t
     const int64_t tiles = (n + kTTileElems - 1) / kTTileElems;
     if (aligned(grad, 16) && aligned(residual, 16)) {
         auto k = quantize_ternary_kernel<true>;
-        k<<<warps_grid(tiles, resident_blocks(k, kThreads, occ_tq[1])), kThreads, 0, stream>>>(
+        k<<<warps_grid(tiles, resident_blocks(k, kThreads, occ_tq[1]), kTernaryQuantizeWaves), kThreads,
+            0, stream>>>(
             grad, residual, compr, n, neg_threshold, pos_threshold);
     } else {
         auto k = quantize_ternary_kernel<false>;
-        k<<<warps_grid(tiles, resident_blocks(k, kThreads, occ_tq[0])), kThreads, 0, stream>>>(
+        k<<<warps_grid(tiles, resident_blocks(k, kThreads, occ_tq[0]), kTernaryQuantizeWaves), kThreads,
+            0, stream>>>(
             grad, residual, compr, n, neg_threshold, pos_threshold);
     }
     return launch_status();
