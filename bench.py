@@ -520,6 +520,18 @@ def time_rows(dev, stream, peak, reps=20, scale=1):
                                                      workload="BERT-Base bucket, 4 workers")
     del keep, comprs, out, tables
 
+    # the single-tensor bf16 quantize on one flat gradient of the bucket's size
+    gb = workloads.normal(total, wb.scale, torch.Generator(device=dev).manual_seed(7), dev,
+                          dtype=torch.bfloat16)
+    rb = torch.zeros(total, device=dev)
+    cb = torch.empty(q.qga_2bit_words(total), dtype=torch.int32, device=dev)
+    t = _time_launches(stream, lambda: ok(L.qga_quantize_2bit_bf16(
+        vp(gb.data_ptr()), vp(rb.data_ptr()), vp(cb.data_ptr()), total, neg[0], pos[0], sp),
+        "quantize_bf16"), reps)
+    rows["quantize_2bit_bf16"] = _row(t, total, 10.25, peak, reps + 3,
+                                      workload=f"one flat bf16 gradient, n={total:,}")
+    del gb, rb, cb
+
     # QSGD-MaxNorm: max over 8 workers, quantize per b, merge of 8
     wq = workloads.WORKLOADS["qsgd-128M-8w"]
     nq, Wq = wq.n // scale, wq.workers
