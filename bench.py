@@ -46,7 +46,7 @@ FALLBACK_HBM_GBS = 6650.0
 # launch of the quantize kernel (profiles/quantize_2bit_kernel_fp32_vgg16.md),
 # keyed by the hash of the sources that kernel is compiled from; reported as
 # null once they have changed since the capture.
-MEASURED_TRAFFIC = {"9a7d18341a8cc830": 11.900}   # 1.6465 GB per launch of n = 138,357,544
+MEASURED_TRAFFIC = {"f3512afac11d18eb": 11.900}   # 1.6465 GB per launch of n = 138,357,544
 QUANT_SOURCES = ("qga_common.cuh", "qga_2bit_tiles.cuh", "qga_2bit.cu")
 
 
@@ -68,15 +68,41 @@ def parse_args():
     return p.parse_args()
 
 
+def _code_only(text):
+    """C/C++ source without its comments and blank lines: the part that can
+    change a kernel (string and character literals are kept as they are)."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            i = text.find("\n", i)
+            i = n if i < 0 else i
+        elif text.startswith("/*", i):
+            i = text.find("*/", i + 2)
+            i = n if i < 0 else i + 2
+        else:
+            out.append(c)
+            i += 1
+    lines = [ln.rstrip() for ln in "".join(out).splitlines()]
+    return "\n".join(ln for ln in lines if ln)
+
+
 def csrc_hash(names=None):
-    """Hash of the CUDA sources (all of them, or the named files)."""
+    """Hash of the CUDA sources' code, comments excluded (all files, or the
+    named ones): it changes exactly when a kernel may have changed."""
     h = hashlib.sha256()
     pkg = os.path.join(ROOT, "quantized_gradient_aggregation_b200", "csrc")
     paths = sorted(glob.glob(os.path.join(pkg, "*.cu*"))) if names is None else \
         [os.path.join(pkg, x) for x in names]
     for path in paths:
-        with open(path, "rb") as f:
-            h.update(f.read())
+        with open(path, encoding="utf-8") as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -6,9 +6,10 @@
 // gradient" (header [neg, pos, n] then 16 codes per word) and "Local kvstore"
 // (the receiver dequantizes every worker's gradient and sums them).
 //
-// Each kernel is one pass over HBM with a persistent grid (every SM filled
-// once; warps stride over tiles: 512 elements for an fp32 quantize or a
-// dequantize, 1024 for a bf16 quantize or a merge slice).  Nothing is filled
+// Each kernel is one pass over HBM: warps stride over tiles (512 elements
+// for an fp32 quantize or a dequantize, 1024 for a bf16 quantize or a merge
+// slice) on a grid of a few waves of resident blocks, the count measured
+// best for each kernel (see grid_for).  Nothing is filled
 // or cleared by a separate launch: the quantize kernel writes every payload
 // word (including the zero tail codes) and its block 0 writes the header.
 // The merge's occupancy and words per lane are build-time settings

@@ -11,7 +11,7 @@
 // every chunk; a tensor of n = 0 still owns one quantizer chunk, which writes
 // its header).  The host numbers the chunks of all tensors consecutively and
 // passes the descriptor table BY VALUE as a kernel parameter (no device
-// table, no allocation, no copy): a persistent grid strides over the chunk
+// table, no allocation, no copy): the grid strides over the chunk
 // numbers, and each block finds its tensor by a binary search over the
 // table's first-chunk column.  Tables over 256 tensors are split into
 // several launches.
