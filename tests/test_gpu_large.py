@@ -101,3 +101,63 @@ def test_qsgd_past_2_31(big):
             got[int(k) * per + i] = d - (1 << b) if d >= (1 << (b - 1)) else d
     for e, gv in zip(elems, g_s):
         assert got[int(e)] == oracle.qsgd_level(gv, Mf, b, 77, int(e)), int(e)
+
+
+def test_fused_reducing_step_past_2_31(big):
+    """The reducing worker's fused quantize + merge at n = 2^31 + 37: its own
+    record words, residuals and the merged values at sampled words near 0,
+    around 2^31 and at the ragged end, against the oracle."""
+    q = qga()
+    g = big
+    words = q.qga_2bit_words(N)
+    pick = _pick(words - 3)
+    spans = [(int(k) * 16, min(int(k) * 16 + 16, N)) for k in pick]
+    other_thr, own_thr = (-1.0, 0.75), (-0.5, 0.5)
+    # worker 0: a record made by the plain quantize (its words are checked there)
+    r0 = torch.zeros(N, device=DEV)
+    c0 = torch.empty(words, dtype=torch.int32, device=DEV)
+    q.qga_quantize_2bit(g, r0, c0, *other_thr)
+    del r0
+    # worker 1 reduces: its own quantize (residual starts at 0) + the merge of both
+    r1 = torch.zeros(N, device=DEV)
+    c1 = torch.empty(words, dtype=torch.int32, device=DEV)
+    out = torch.empty(N, device=DEV)
+    q.qga_quantize_merge_2bit(g, r1, [c0, c1], 1, *own_thr, out)
+    g_s, _ = gather_elems(g, pick, 16, N)
+    r_s, _ = gather_elems(r1, pick, 16, N)
+    o_s, _ = gather_elems(out, pick, 16, N)
+    got1 = u32(c1.index_select(0, torch.from_numpy(pick + 3).to(DEV)))
+    g_s, r_s, o_s = g_s.numpy(), r_s.numpy(), o_s.numpy()
+    at = 0
+    for i, (a, b) in enumerate(spans):
+        m = b - a
+        w0, _ = oracle.quantize_2bit(g_s[at:at + m], np.zeros(m, np.float32), *other_thr)
+        w1, wr = oracle.quantize_2bit(g_s[at:at + m], np.zeros(m, np.float32), *own_thr)
+        assert got1[i] == w1[3], int(pick[i])
+        assert same_bits_f32(r_s[at:at + m], wr), int(pick[i])
+        want = oracle.dequant_accumulate_2bit([w0, w1], m)
+        assert same_bits_f32(o_s[at:at + m], want), int(pick[i])
+        at += m
+    del r1, c1, c0, out
+
+
+def test_grandk_coordinates_past_2_31(big):
+    """GRandK-MaxNorm with kept coordinates on both sides of 2^31."""
+    q = qga()
+    g = big
+    rng = np.random.default_rng(3)
+    index = np.unique(np.concatenate([rng.integers(0, N, 600), (1 << 31) + np.arange(-20, 20),
+                                      [N - 1, 0]])).astype(np.int64)
+    rng.shuffle(index)
+    idx = torch.from_numpy(index).to(DEV)
+    M = torch.empty(1, device=DEV)
+    q.qga_grandk_mn_max([g], idx, M)
+    kept = f32(g.index_select(0, idx))
+    ident = np.arange(index.size, dtype=np.int64)
+    want_M = oracle.grandk_mn_max([kept], ident)
+    assert M.item() == want_M
+    for b in (2, 8):
+        c = torch.empty(q.qga_qsgd_words(index.size, b), dtype=torch.int32, device=DEV)
+        q.qga_grandk_mn_quantize(g, idx, c, b, 99, M)
+        want = oracle.grandk_mn_quantize(kept, ident, b, 99, want_M)
+        assert np.array_equal(u32(c), want), b
