@@ -626,12 +626,12 @@ def time_rows(dev, stream, peak, reps=20, scale=1):
 
 def run_e2e(args, w, dev_grads, res, comprs, out, quant, reduce, stream, world, dev):
     """Same step with the gradients arriving from pinned host memory and the
-    aggregate read back, copies inside the timed region.  Copies run on a
-    second stream: worker k's upload overlaps the quantize of the worker
-    before it, and the aggregate's download (the other PCIe direction)
-    overlaps the next step's uploads; events order every reuse of a buffer.
-    Worker 0, the reducing worker, comes last: its quantize and the merge
-    are one launch."""
+    aggregate read back, copies inside the timed region.  Uploads run on one
+    copy stream, so worker k's upload overlaps the quantize of the worker
+    before it; the aggregate's download runs on another, so that it overlaps
+    the next step's uploads (PCIe carries both directions at once).  Events
+    order every reuse of a buffer.  Worker 0, the reducing worker, comes
+    last: its quantize and the merge are one launch."""
     import torch
     n, W = w.n, w.workers
     host = [torch.empty(n, dtype=torch.float32, pin_memory=True) for _ in range(W)]
@@ -639,6 +639,7 @@ def run_e2e(args, w, dev_grads, res, comprs, out, quant, reduce, stream, world, 
         host[k].copy_(dev_grads[k], non_blocking=False)
     host_out = torch.empty(n, dtype=torch.float32, pin_memory=True)
     copy_stream = torch.cuda.Stream(device=dev)
+    down_stream = torch.cuda.Stream(device=dev)
     K = max(3, min(args.steps, 10))
     landed = [torch.cuda.Event() for _ in range(W)]
     consumed = [torch.cuda.Event() for _ in range(W)]
@@ -662,10 +663,10 @@ def run_e2e(args, w, dev_grads, res, comprs, out, quant, reduce, stream, world, 
                 reduce(0)
                 merged.record(stream)
             consumed[k].record(stream)
-        with torch.cuda.stream(copy_stream):
-            copy_stream.wait_event(merged)
+        with torch.cuda.stream(down_stream):
+            down_stream.wait_event(merged)
             host_out.copy_(out, non_blocking=True)
-            downloaded.record(copy_stream)
+            downloaded.record(down_stream)
 
     for _ in range(2):
         step()
@@ -685,7 +686,7 @@ def run_e2e(args, w, dev_grads, res, comprs, out, quant, reduce, stream, world, 
     return {"value": job_gelem_per_s(world, W, n, K, ms), "unit": "Gelem/s",
             "h2d_bytes_per_step": W * n * 4, "d2h_bytes_per_step": n * 4, "steps": K,
             "path": "pinned host gradients -> cudaMemcpyAsync (copy stream) -> qga_quantize_2bit x7 "
-                    "-> qga_quantize_merge_2bit (worker 0) -> pinned host aggregate (copy stream)"}
+                    "-> qga_quantize_merge_2bit (worker 0) -> pinned host aggregate (download stream)"}
 
 
 def main():
