@@ -46,7 +46,7 @@ FALLBACK_HBM_GBS = 6650.0
 # launch of the quantize kernel (profiles/quantize_2bit_kernel_fp32_vgg16.md),
 # keyed by the hash of the sources that kernel is compiled from; reported as
 # null once they have changed since the capture.
-MEASURED_TRAFFIC = {"f3512afac11d18eb": 11.900}   # 1.6465 GB per launch of n = 138,357,544
+MEASURED_TRAFFIC = {"f29bd18f50f18594": 11.871}   # 1.6425 GB per launch of n = 138,357,544
 QUANT_SOURCES = ("qga_common.cuh", "qga_2bit_tiles.cuh", "qga_2bit.cu")
 
 
@@ -391,7 +391,7 @@ def run_qga(args, rank, world, local_rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded Laplace(0,1e-3) gradients generated on the GPU)",
         "config": workload_config(w, world),
-        "roofline": {"bound": "hbm", "kernel": "qga_quantize_2bit (quantize_2bit_kernel<float>)",
+        "roofline": {"bound": "hbm", "kernel": "qga_quantize_2bit (quantize_2bit_words_kernel)",
                      "achieved": quant_gbs, "peak": peak, "unit": "GB/s", "frac": quant_gbs / peak,
                      "peak_source": f"{peak_kind} HBM copy rate",
                      "bytes_per_elem": QUANT_BYTES_PER_ELEM, "elems_per_launch": n,

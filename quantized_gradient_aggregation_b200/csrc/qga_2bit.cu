@@ -43,6 +43,30 @@ __global__ void __launch_bounds__(kThreads)
         quantize_2bit_tile<G, kVec>(grad, residual, compr + 3, n, t, neg, pos, lane);
 }
 
+// fp32 quantize in lane-owned words (gradient and residual 32-byte aligned):
+// warp t of the grid owns words 32 t .. 32 t + 31, one per lane.
+__global__ void __launch_bounds__(kThreads)
+    quantize_2bit_words_kernel(const float *__restrict__ grad, float *__restrict__ residual,
+                               uint32_t *__restrict__ compr, int64_t n, float neg, float pos)
+{
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        compr[0] = bits_from_f32(neg);
+        compr[1] = bits_from_f32(pos);
+        compr[2] = bits_from_f32(__ll2float_rn(n));
+    }
+    const int lane = threadIdx.x & (kWarp - 1);
+    const int64_t nwords = (n + 15) >> 4;
+    const int64_t runs = (nwords + kWarp - 1) / kWarp;
+    for (int64_t t = first_tile(); t < runs; t += tile_stride()) {
+        const int64_t k = t * kWarp + lane;
+        if (k < nwords) {
+            float g[16], r[16];
+            load_word<true>(grad, residual, n, k, g, r);
+            quantize_word<true>(residual, compr + 3, n, k, neg, pos, g, r);
+        }
+    }
+}
+
 template <bool kVec>
 __global__ void __launch_bounds__(kThreads)
     dequantize_2bit_kernel(const uint32_t *__restrict__ compr, float *__restrict__ out, int64_t n)
@@ -98,14 +122,15 @@ __global__ void __launch_bounds__(kThreads, QGA_MERGE_MIN_BLOCKS)
     }
 }
 
-std::atomic<int> occ_q_f32_v[64], occ_q_f32_s[64], occ_q_bf16_v[64], occ_q_bf16_s[64];
+std::atomic<int> occ_q_f32_w[64], occ_q_f32_v[64], occ_q_f32_s[64], occ_q_bf16_v[64], occ_q_bf16_s[64];
 std::atomic<int> occ_dq_v[64], occ_dq_s[64];
 std::atomic<int> occ_acc[2][9][64]; // [vec][kW][device]
 
-// Grid waves (see grid_for), measured at n = 138M: quantize 1 / 8 / 16 / 32 /
-// 128 waves 270-286 / 263 / 259 / 256 / 258 us; dequantize 109 / 97 / 96 /
-// 101 us at 1 / 8 / 16 / 32; merge (W = 8) 180 / 174 / 176 / 181 us at
-// 1 / 8 / 16 / 32.
+// Grid waves (see grid_for), measured at n = 138M: quantize in group tiles
+// 270-286 / 263 / 259 / 256 / 258 us at 1 / 8 / 16 / 32 / 128 waves, in
+// lane-owned words 252 / 243 us at 8 / 32 waves (2 words per lane: 253 /
+// 256); dequantize 109 / 97 / 96 / 101 us at 1 / 8 / 16 / 32; merge (W = 8)
+// 180 / 174 / 176 / 181 us at 1 / 8 / 16 / 32.
 constexpr int kQuantizeWaves = 32, kDequantizeWaves = 16, kMergeWaves = 8;
 
 unsigned tiles_grid(int64_t n, int resident, int64_t elems_per_warp, int waves)
@@ -149,7 +174,8 @@ void launch_merge(const RecordSet &set, int W, float *out, int64_t n, cudaStream
 
 template <typename G>
 int launch_quantize(const G *grad, float *residual, uint32_t *compr, int64_t n, float neg, float pos,
-                    cudaStream_t stream, std::atomic<int> *occ_v, std::atomic<int> *occ_s)
+                    cudaStream_t stream, std::atomic<int> *occ_v, std::atomic<int> *occ_s,
+                    std::atomic<int> *occ_w = nullptr)
 {
     if (n < 0 || compr == nullptr || !aligned(compr, 4) || !finite_f32(neg) || !finite_f32(pos))
         return QGA_ERR_INVALID_ARG;
@@ -158,6 +184,14 @@ int launch_quantize(const G *grad, float *residual, uint32_t *compr, int64_t n, 
         return QGA_ERR_INVALID_ARG;
     const bool vec = aligned(grad, GradLoad<G>::kVecAlign) && aligned(residual, 16);
     constexpr int64_t kElems = quantize_tile_elems<G>();
+    if constexpr (sizeof(G) == sizeof(float)) {
+        if (aligned(grad, 32) && aligned(residual, 32)) {
+            auto k = quantize_2bit_words_kernel;
+            k<<<tiles_grid(n, resident_blocks(k, kThreads, occ_w), 16 * kWarp, kQuantizeWaves),
+                kThreads, 0, stream>>>(grad, residual, compr, n, neg, pos);
+            return launch_status();
+        }
+    }
     if (vec) {
         auto k = quantize_2bit_kernel<G, true>;
         k<<<tiles_grid(n, resident_blocks(k, kThreads, occ_v), kElems, kQuantizeWaves), kThreads, 0,
@@ -188,7 +222,7 @@ extern "C" int qga_quantize_2bit(const float *grad, float *residual, uint32_t *c
                                  float neg_threshold, float pos_threshold, cudaStream_t stream)
 {
     return launch_quantize<float>(grad, residual, compr, n, neg_threshold, pos_threshold, stream,
-                                  occ_q_f32_v, occ_q_f32_s);
+                                  occ_q_f32_v, occ_q_f32_s, occ_q_f32_w);
 }
 
 extern "C" int qga_quantize_2bit_bf16(const uint16_t *grad, float *residual, uint32_t *compr,

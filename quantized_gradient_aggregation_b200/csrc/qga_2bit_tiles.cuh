@@ -166,6 +166,65 @@ __device__ __forceinline__ void quantize_2bit_tile(const G *__restrict__ grad,
     }
 }
 
+// ---------------------------------------------------- lane-owned words --
+// The other geometry for an fp32 gradient whose gradient and residual are
+// 32-byte aligned: a lane owns whole words (16 consecutive elements), loads
+// them with two 256-bit loads each of g and r, packs its 16 codes in
+// registers (no shuffle) and stores r with two 256-bit stores.  Each warp
+// access still uses whole 32-byte sectors, with a quarter of the memory
+// instructions of the group tiles.  load_word and quantize_word are its two
+// halves (the loads of several words can be issued before any is used).
+// Codes of elements >= n are 00.
+template <bool kVec>
+__device__ __forceinline__ void load_word(const float *__restrict__ grad,
+                                          const float *__restrict__ residual, int64_t n,
+                                          int64_t k, float (&g)[16], float (&r)[16])
+{
+    const int64_t e0 = 16 * k;
+    if (kVec && e0 + 16 <= n) {
+        ld_stream_f8(grad + e0, g);
+        ld_stream_f8(grad + e0 + 8, g + 8);
+        ld_stream_f8(residual + e0, r);
+        ld_stream_f8(residual + e0 + 8, r + 8);
+    } else {
+#pragma unroll
+        for (int p = 0; p < 16; ++p) {
+            g[p] = e0 + p < n ? ld_stream_f1(grad + e0 + p) : 0.0f;
+            r[p] = e0 + p < n ? ld_stream_f1(residual + e0 + p) : 0.0f;
+        }
+    }
+}
+
+// Codes and residual update of word k from its loaded elements; writes the
+// residual and the word, and returns the word.
+template <bool kVec>
+__device__ __forceinline__ uint32_t quantize_word(float *__restrict__ residual,
+                                                  uint32_t *__restrict__ payload, int64_t n,
+                                                  int64_t k, float neg, float pos,
+                                                  const float (&g)[16], float (&r)[16])
+{
+    const int64_t e0 = 16 * k;
+    const bool full = kVec && e0 + 16 <= n;
+    uint32_t word = 0u;
+#pragma unroll
+    for (int p = 0; p < 16; ++p) {
+        const uint32_t c = tb_step(g[p], r[p], neg, pos);
+        if (full || e0 + p < n)
+            word |= c << (30 - 2 * p);
+    }
+    if (full) {
+        st_stream_f8(residual + e0, r);
+        st_stream_f8(residual + e0 + 8, r + 8);
+    } else {
+#pragma unroll
+        for (int p = 0; p < 16; ++p)
+            if (e0 + p < n)
+                st_stream_f1(residual + e0 + p, r[p]);
+    }
+    st_stream_u32(payload + k, word);
+    return word;
+}
+
 // Values of the 4 codes in a byte (first element in bits 7..6).
 __device__ __forceinline__ float4 tb_decode4(uint32_t byte, float neg, float pos)
 {

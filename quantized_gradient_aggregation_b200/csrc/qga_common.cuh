@@ -69,6 +69,15 @@ __device__ __forceinline__ void st_stream_f4(float *p, float4 v)
                  : "memory");
 }
 
+// 256-bit streaming load (sm_100): p must be 32-byte aligned.
+__device__ __forceinline__ void ld_stream_f8(const float *p, float *v)
+{
+    asm volatile("ld.global.cs.L2::256B.v8.f32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]),
+                   "=f"(v[6]), "=f"(v[7])
+                 : "l"(p));
+}
+
 // 256-bit store (sm_100): p must be 32-byte aligned.
 __device__ __forceinline__ void st_stream_f8(float *p, const float *v)
 {

@@ -36,7 +36,9 @@ constexpr int kWarpsPerBlock = kThreads / kWarp;
 // 496 us.  Issuing both words' loads before either is quantized (470-618 us)
 // and prefetching the next slice into L2 (570-602 us) were slower; issuing
 // the received records' loads before the own quantize changed nothing
-// (426 us, at 3 blocks to avoid spills).
+// (426 us, at 3 blocks to avoid spills).  More grid waves: 426 / 440 us at 8
+// / 32; with one word per lane in the merge slice 432 / 411 / 424 us at 1 /
+// 8 / 32 waves (that slice width is shared with the plain and bucket merges).
 #ifndef QGA_LOCAL_REDUCE_MIN_BLOCKS
 #define QGA_LOCAL_REDUCE_MIN_BLOCKS 4
 #endif
@@ -44,67 +46,6 @@ constexpr int kWarpsPerBlock = kThreads / kWarp;
 struct RecordSet {
     const uint32_t *rec[QGA_MAX_WORKERS];
 };
-
-// 256-bit streaming load (sm_100): p must be 32-byte aligned.
-__device__ __forceinline__ void ld_stream_f8(const float *p, float *v)
-{
-    asm volatile("ld.global.cs.L2::256B.v8.f32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                 : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]),
-                   "=f"(v[6]), "=f"(v[7])
-                 : "l"(p));
-}
-
-// Quantize + residual update + pack of word k (elements 16k .. 16k+15) of
-// the own gradient, in two halves so that a lane can have the loads of
-// several words in flight: load_word, then quantize_word.  Codes of
-// elements >= n are 00.
-//   kVec: grad and residual are 32-byte aligned.
-template <bool kVec>
-__device__ __forceinline__ void load_word(const float *__restrict__ grad,
-                                          const float *__restrict__ residual, int64_t n,
-                                          int64_t k, float (&g)[16], float (&r)[16])
-{
-    const int64_t e0 = 16 * k;
-    if (kVec && e0 + 16 <= n) {
-        ld_stream_f8(grad + e0, g);
-        ld_stream_f8(grad + e0 + 8, g + 8);
-        ld_stream_f8(residual + e0, r);
-        ld_stream_f8(residual + e0 + 8, r + 8);
-    } else {
-#pragma unroll
-        for (int p = 0; p < 16; ++p) {
-            g[p] = e0 + p < n ? ld_stream_f1(grad + e0 + p) : 0.0f;
-            r[p] = e0 + p < n ? ld_stream_f1(residual + e0 + p) : 0.0f;
-        }
-    }
-}
-
-template <bool kVec>
-__device__ __forceinline__ void quantize_word(float *__restrict__ residual,
-                                              uint32_t *__restrict__ payload, int64_t n, int64_t k,
-                                              float neg, float pos, const float (&g)[16],
-                                              float (&r)[16])
-{
-    const int64_t e0 = 16 * k;
-    const bool full = kVec && e0 + 16 <= n;
-    uint32_t word = 0u;
-#pragma unroll
-    for (int p = 0; p < 16; ++p) {
-        const uint32_t c = tb_step(g[p], r[p], neg, pos);
-        if (full || e0 + p < n)
-            word |= c << (30 - 2 * p);
-    }
-    if (full) {
-        st_stream_f8(residual + e0, r);
-        st_stream_f8(residual + e0 + 8, r + 8);
-    } else {
-#pragma unroll
-        for (int p = 0; p < 16; ++p)
-            if (e0 + p < n)
-                st_stream_f1(residual + e0 + p, r[p]);
-    }
-    st_stream_u32(payload + k, word);
-}
 
 // kW > 0: compiled for exactly kW workers; kW == 0: any W up to QGA_MAX_WORKERS.
 template <bool kVec, int kW>

@@ -69,7 +69,10 @@ def test_quantize_fp32_ragged(n, thr):
 
 
 @pytest.mark.parametrize("n", [1, 17, 513, 4097, 65_537])
-@pytest.mark.parametrize("offsets", [(1, 0, 0), (0, 1, 0), (0, 0, 1), (3, 2, 1)])
+@pytest.mark.parametrize("offsets", [(1, 0, 0), (0, 1, 0), (0, 0, 1), (3, 2, 1),
+                                     # 16- but not 32-byte aligned (group tiles), then
+                                     # both 32-byte aligned at an offset (lane-owned words)
+                                     (4, 4, 0), (4, 0, 0), (8, 8, 3)])
 def test_quantize_fp32_misaligned(n, offsets):
     og, orr, oc = offsets
     g0, r0 = _inputs(n, 7 + n)
