@@ -80,9 +80,8 @@ static uint32_t two_bit_code(float value, float neg_thr, float pos_thr)
 }
 
 /* Value a code stands for: the threshold that produced it, or zero.  The
- * header keeps the thresholds because they "are required to dequantize"
- * ([MX] "Format of compressed gradient").  Code 11 is never produced; it
- * decodes to zero. */
+ * header keeps the thresholds because decoding needs them ([MX] "Format of
+ * compressed gradient").  Code 11 is never produced; it decodes to zero. */
 static float two_bit_value(uint32_t code, float neg_thr, float pos_thr)
 {
     if (code == 1u)

@@ -4,7 +4,8 @@
 // MXNet pull request #8342 "[WIP] 2bit gradient compression", "Local
 // kvstore": the device that sums the gradients dequantizes every worker's
 // compressed gradient and merges them, and it also quantizes (and so
-// error-feeds) its own gradient, "so that there is no bias" ("Questions", 1).
+// error-feeds) its own gradient, so that its own samples are treated like
+// every other worker's (the page's reason, and its "Questions", 1).
 // Done as two calls, that device's own quantize writes its record and the
 // merge reads it straight back.  Here one kernel does both: a warp quantizes
 // the words of its slice of the own gradient (residual updated, record words
