@@ -46,11 +46,17 @@ class CompressedAllGather:
     (updated in place) with the thresholds given here, all-gathers the
     records of the ``group``'s ranks and writes their merge (worker order =
     rank order) into ``out``.  The two record buffers are allocated once,
-    here, on the current CUDA device.
+    here, on ``device`` (default: the current CUDA device).
+
+    ``ops`` replaces the format's three library calls by a triple
+    ``(words(n), quantize(grad, residual, compr, neg, pos), merge(records,
+    out))`` with the same arguments; it exists so that the step's ordering
+    (quantize, gather, merge in rank order, residual carried) can be driven
+    on a CPU process group with stand-in arithmetic.
     """
 
     def __init__(self, n: int, neg_threshold: float, pos_threshold: float, group=None,
-                 fmt: str = "2bit"):
+                 fmt: str = "2bit", *, device=None, ops=None):
         if fmt not in _FORMATS:
             raise ValueError(f"format {fmt!r}: one of {sorted(_FORMATS)}")
         self.n = int(n)
@@ -58,9 +64,10 @@ class CompressedAllGather:
         self.pos = float(pos_threshold)
         self.group = group
         self.world = dist.get_world_size(group)
-        words_fn, self._quantize, self._merge = _FORMATS[fmt]
+        words_fn, self._quantize, self._merge = _FORMATS[fmt] if ops is None else ops
         self.words = int(words_fn(self.n))
-        device = torch.device("cuda", torch.cuda.current_device())
+        if device is None:
+            device = torch.device("cuda", torch.cuda.current_device())
         self.local = torch.empty(self.words, dtype=torch.int32, device=device)
         self.gathered = torch.empty(self.world * self.words, dtype=torch.int32, device=device)
 
@@ -80,18 +87,31 @@ class BucketedCompressedAllGather:
     per-tensor thresholds.  ``step(grads, residuals, outs)`` takes per bucket
     the gradient tensors (fp32 or bf16, one dtype per bucket), the fp32
     residuals (updated in place) and one flat fp32 output holding the
-    bucket's merged tensors one after the other.
+    bucket's merged tensors one after the other.  Record buffers live on
+    ``device`` (default: the current CUDA device).
+
+    ``ops`` replaces the four library calls by ``(words(sizes),
+    make_table(grads, residuals, neg, pos), quantize(grads, residuals, neg,
+    pos, compr, table=...), merge(records, sizes, out))`` with the same
+    arguments, so that the pipeline's ordering can be driven on a CPU
+    process group with stand-in arithmetic.
     """
 
-    def __init__(self, buckets, neg, pos, group=None):
-        from . import qga_2bit_bucket_words
+    def __init__(self, buckets, neg, pos, group=None, *, device=None, ops=None):
+        from . import (make_bucket_table, qga_2bit_bucket_words, qga_dequant_accumulate_2bit_bucket,
+                       qga_quantize_2bit_bucket)
+        if ops is None:
+            ops = (qga_2bit_bucket_words, make_bucket_table, qga_quantize_2bit_bucket,
+                   qga_dequant_accumulate_2bit_bucket)
+        words_fn, self._make_table, self._quantize, self._merge = ops
         self.sizes = [list(map(int, b)) for b in buckets]
         self.neg = [list(map(float, x)) for x in neg]
         self.pos = [list(map(float, x)) for x in pos]
         self.group = group
         self.world = dist.get_world_size(group)
-        device = torch.device("cuda", torch.cuda.current_device())
-        self.words = [qga_2bit_bucket_words(s) for s in self.sizes]
+        if device is None:
+            device = torch.device("cuda", torch.cuda.current_device())
+        self.words = [int(words_fn(s)) for s in self.sizes]
         self.local = [torch.empty(w, dtype=torch.int32, device=device) for w in self.words]
         self.gathered = [torch.empty(self.world * w, dtype=torch.int32, device=device)
                          for w in self.words]
@@ -102,22 +122,20 @@ class BucketedCompressedAllGather:
         return list(self.gathered[b].view(self.world, self.words[b]).unbind(0))
 
     def step(self, grads, residuals, outs) -> None:
-        from . import (make_bucket_table, qga_dequant_accumulate_2bit_bucket,
-                       qga_quantize_2bit_bucket)
         key = tuple((g.data_ptr(), r.data_ptr()) for bg, br in zip(grads, residuals)
                     for g, r in zip(bg, br))
         if key != self._table_key:  # descriptor tables: rebuilt only when a buffer moved
-            self._tables = [make_bucket_table(grads[b], residuals[b], self.neg[b], self.pos[b])
+            self._tables = [self._make_table(grads[b], residuals[b], self.neg[b], self.pos[b])
                             for b in range(len(self.sizes))]
             self._table_key = key
         works = []
         for b in range(len(self.sizes)):
-            qga_quantize_2bit_bucket(grads[b], residuals[b], self.neg[b], self.pos[b],
-                                     self.local[b], table=self._tables[b])
+            self._quantize(grads[b], residuals[b], self.neg[b], self.pos[b], self.local[b],
+                           table=self._tables[b])
             # NCCL orders the collective after the work already on the current
             # stream, and runs it beside the next bucket's quantize
             works.append(dist.all_gather_into_tensor(self.gathered[b], self.local[b],
                                                      group=self.group, async_op=True))
         for b, work in enumerate(works):
             work.wait()  # the current stream waits for bucket b's records only
-            qga_dequant_accumulate_2bit_bucket(self.records(b), self.sizes[b], outs[b])
+            self._merge(self.records(b), self.sizes[b], outs[b])

@@ -110,3 +110,123 @@ def test_record_gather_layout_on_two_and_three_ranks():
         """, world=world)
         digests = {o.strip().splitlines()[-1] for o in outs}
         assert len(digests) == 1
+
+
+# The exchange steps end to end on gloo ranks: every rank quantizes its OWN
+# seeded gradient, the records cross the process group, and every rank must
+# hold the merge of all ranks' records in rank order, with its residual
+# carried over three steps.  The arithmetic is the oracle's (injected through
+# the classes' ``ops``, on host tensors); what is under test is the classes'
+# ordering: quantize, gather, merge rows in rank order, buffers reused.
+_EXCHANGE_PRELUDE = """
+    import numpy as np, torch, oracle
+    from quantized_gradient_aggregation_b200.exchange import (
+        BucketedCompressedAllGather, CompressedAllGather)
+
+    def as_u32(t):
+        return t.numpy().view(np.uint32)
+
+    def q2(grad, residual, compr, neg, pos):
+        c, r = oracle.quantize_2bit(grad.numpy(), residual.numpy(), neg, pos)
+        compr.copy_(torch.from_numpy(c.view(np.int32)))
+        residual.copy_(torch.from_numpy(r))
+
+    def m2(records, out):
+        out.copy_(torch.from_numpy(oracle.dequant_accumulate_2bit(
+            [as_u32(r) for r in records], out.numel())))
+
+    def qt(grad, residual, compr, neg, pos):
+        c, r = oracle.quantize_ternary(grad.numpy(), residual.numpy(), neg, pos)
+        compr.copy_(torch.from_numpy(c.view(np.int32)))
+        residual.copy_(torch.from_numpy(r))
+
+    def mt(records, out):
+        out.copy_(torch.from_numpy(oracle.dequant_accumulate_ternary(
+            [as_u32(r) for r in records], out.numel())))
+
+    def grad_of(rank_, step, n):
+        g = np.random.default_rng(1000 * rank_ + step).standard_normal(n) * 0.4
+        return g.astype(np.float32)
+"""
+
+
+@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("fmt", ["2bit", "ternary"])
+def test_exchange_step_distinct_ranks(world, fmt):
+    outs = _run_ranks(_EXCHANGE_PRELUDE + f"""
+    fmt = {fmt!r}
+    n, neg, pos = 10_007, -0.25, 0.25
+    ops = (oracle.words_2bit, q2, m2) if fmt == "2bit" else (oracle.words_ternary, qt, mt)
+    quant = oracle.quantize_2bit if fmt == "2bit" else oracle.quantize_ternary
+    merge = oracle.dequant_accumulate_2bit if fmt == "2bit" else oracle.dequant_accumulate_ternary
+    ex = CompressedAllGather(n, neg, pos, fmt=fmt, device="cpu", ops=ops)
+    r = torch.zeros(n)
+    out = torch.empty(n)
+    res_all = [np.zeros(n, np.float32) for _ in range(world)]
+    for step in range(3):
+        ex.step(torch.from_numpy(grad_of(rank, step, n)), r, out)
+        recs = []
+        for k in range(world):  # every rank's record, recomputed from its seed
+            c, res_all[k] = quant(grad_of(k, step, n), res_all[k], neg, pos)
+            recs.append(c)
+        rows = as_u32(ex.gathered).reshape(world, -1)
+        for k in range(world):
+            assert np.array_equal(rows[k], recs[k]), (step, k)
+        assert np.array_equal(r.numpy().view(np.uint32), res_all[rank].view(np.uint32)), step
+        want = merge(recs, n)
+        assert np.array_equal(out.numpy().view(np.uint32), want.view(np.uint32)), step
+    assert len({{bytes(as_u32(ex.gathered))}}) == 1
+    print("ok", float(out.abs().sum()))
+    """, world=world)
+    sums = {o.strip().splitlines()[-1] for o in outs}
+    assert len(sums) == 1 and next(iter(sums)).startswith("ok")
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_bucketed_exchange_distinct_ranks(world):
+    outs = _run_ranks(_EXCHANGE_PRELUDE + """
+    buckets = [[768, 3072, 4099, 17], [3000, 5, 768 * 4]]
+    neg = [[-2e-3] * len(b) for b in buckets]
+    pos = [[2e-3 + 1e-4 * i for i in range(len(b))] for b in buckets]
+
+    def qb(grads, residuals, neg_, pos_, compr, table=None):
+        assert table == ("table", len(grads))
+        c, rs = oracle.quantize_2bit_bucket([g.numpy() for g in grads],
+                                            [r.numpy() for r in residuals], neg_, pos_)
+        compr.copy_(torch.from_numpy(c.view(np.int32)))
+        for r, new in zip(residuals, rs):
+            r.copy_(torch.from_numpy(new))
+
+    def mb(records, sizes, out):
+        out.copy_(torch.from_numpy(oracle.dequant_accumulate_2bit_bucket(
+            [as_u32(r) for r in records], sizes)))
+
+    ops = (oracle.bucket_words_2bit, lambda g, r, a, b: ("table", len(g)), qb, mb)
+    ex = BucketedCompressedAllGather(buckets, neg, pos, device="cpu", ops=ops)
+
+    def bucket_grads(rank_, step):
+        return [[torch.from_numpy(grad_of(100 * rank_ + 10 * b + t, step, s) * 1e-2)
+                 for t, s in enumerate(sizes)] for b, sizes in enumerate(buckets)]
+
+    res = [[torch.zeros(s) for s in b] for b in buckets]
+    outs_ = [torch.empty(sum(b)) for b in buckets]
+    res_all = [[[np.zeros(s, np.float32) for s in b] for b in buckets] for _ in range(world)]
+    for step in range(3):
+        ex.step(bucket_grads(rank, step), res, outs_)
+        for b, sizes in enumerate(buckets):
+            recs = []
+            for k in range(world):
+                g_k = [x.numpy() for x in bucket_grads(k, step)[b]]
+                c, res_all[k][b] = oracle.quantize_2bit_bucket(g_k, res_all[k][b], neg[b], pos[b])
+                recs.append(c)
+            rows = as_u32(ex.gathered[b]).reshape(world, -1)
+            for k in range(world):
+                assert np.array_equal(rows[k], recs[k]), (step, b, k)
+            want = oracle.dequant_accumulate_2bit_bucket(recs, sizes)
+            assert np.array_equal(outs_[b].numpy().view(np.uint32), want.view(np.uint32)), (step, b)
+            for t in range(len(sizes)):
+                assert np.array_equal(res[b][t].numpy(), res_all[rank][b][t]), (step, b, t)
+    print("ok", sum(float(o.abs().sum()) for o in outs_))
+    """, world=world)
+    sums = {o.strip().splitlines()[-1] for o in outs}
+    assert len(sums) == 1 and next(iter(sums)).startswith("ok")
