@@ -81,6 +81,12 @@ def _declare(L):
     L.oracle_qsgd_mn_quantize.argtypes = [vp, vp, i64, i32, u64, f32]
     L.oracle_qsgd_mn_dequant_accumulate.argtypes = [vp, i32, vp, i64, i32]
     L.oracle_ternary_words.restype = i64
+    L.oracle_qsgd_mnts_words.restype = i64
+    L.oracle_qsgd_mnts_words.argtypes = [i64, i32, i32]
+    L.oracle_qsgd_mnts_fine_scale.restype = f32
+    L.oracle_qsgd_mnts_fine_scale.argtypes = [f32, i32]
+    L.oracle_qsgd_mnts_quantize.argtypes = [vp, vp, i64, i32, i32, u64, f32]
+    L.oracle_qsgd_mnts_dequant_accumulate.argtypes = [vp, i32, vp, i64, i32, i32]
     L.oracle_grandk_mn_max.restype = f32
     L.oracle_grandk_mn_max.argtypes = [vp, i32, i64, vp, i64]
     L.oracle_grandk_mn_quantize.argtypes = [vp, i64, vp, i64, vp, i32, u64, f32]
@@ -222,6 +228,38 @@ def qsgd_mn_dequant_accumulate(comprs, n, b, L=None):
     comprs = [_c(c, np.uint32) for c in comprs]
     out = np.empty(n, np.float32)
     L.oracle_qsgd_mn_dequant_accumulate(_ptr_array(comprs), len(comprs), out.ctypes.data, n, b)
+    return out
+
+
+# ----------------------------------------------------------- QSGD-MN-TS ----
+
+def qsgd_mnts_words(n: int, b1: int, b2: int, L=None) -> int:
+    L = L or lib()
+    return int(L.oracle_qsgd_mnts_words(n, b1, b2))
+
+
+def qsgd_mnts_fine_scale(M, b1: int, L=None) -> np.float32:
+    L = L or lib()
+    return np.float32(L.oracle_qsgd_mnts_fine_scale(float(M), b1))
+
+
+def qsgd_mnts_quantize(grad, b1, b2, seed, M, L=None):
+    """Two-scale record: the coarse QSGD-MaxNorm record of b1 bits, then the
+    fine one of b2 bits."""
+    L = L or lib()
+    grad = _c(grad, np.float32)
+    n = grad.size
+    compr = np.zeros(int(L.oracle_qsgd_mnts_words(n, b1, b2)), np.uint32)
+    L.oracle_qsgd_mnts_quantize(grad.ctypes.data, compr.ctypes.data, n, b1, b2, seed, float(M))
+    return compr
+
+
+def qsgd_mnts_dequant_accumulate(comprs, n, b1, b2, L=None):
+    L = L or lib()
+    comprs = [_c(c, np.uint32) for c in comprs]
+    out = np.empty(n, np.float32)
+    L.oracle_qsgd_mnts_dequant_accumulate(_ptr_array(comprs), len(comprs), out.ctypes.data, n,
+                                          b1, b2)
     return out
 
 

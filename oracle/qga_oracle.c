@@ -23,7 +23,9 @@
  *         s = 2^(b-1)-1 levels, stochastic rounding, signed b-bit codes).
  *         "Results" also names GlobalRandKMaxNorm compression (K = 10000) as
  *         its sparsified variant, again without a formula; the GRandK-MN
- *         functions state this library's reading of it.
+ *         functions state this library's reading of it.  It names the
+ *         two-scale QSGDMaxNormMultiScale variant (QSGD-MN-TS) the same way;
+ *         the QSGD-MN-TS functions state this library's reading of that.
  *   [SC11] J. Salmon, M. Moraes, R. Dror, D. Shaw, "Parallel Random Numbers:
  *         As Easy as 1, 2, 3", SC'11 -- the Philox4x32-10 generator.
  *
@@ -372,6 +374,85 @@ void oracle_qsgd_mn_dequant_accumulate(const uint32_t *const *compr, int W, floa
         for (int w = 0; w < W; ++w)
             sum += qsgd_level_at(compr[w], e, b);
         out[e] = (float)sum * step;
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* QSGD-MaxNorm with two scales (QSGD-MN-TS)                           */
+/* ------------------------------------------------------------------ */
+/* [GC] "Results" names QSGDMaxNormMultiScale quantization run with two
+ * scales (TS) of compression, each run labelled with the bit widths of its
+ * two scales, and gives no formula; [GC] "About The Project" counts it among
+ * the all-reduce compatible schemes.  This library's reading:
+ *   - the coarse scale is the QSGD-MaxNorm scale M1 = M (the global max |g|)
+ *     with b1 bits, s1 = 2^(b1-1) - 1 levels;
+ *   - the fine scale is the coarse grid's first step, M2 = M1 / s1 (one
+ *     binary32 division), with b2 bits, s2 = 2^(b2-1) - 1 levels;
+ *   - an element with |g| <= M2 takes the fine scale, any other element the
+ *     coarse one: its level is the QSGD-MaxNorm level with that scale's M and
+ *     s and the element's own draw; its level on the other scale is 0;
+ *   - the record is the coarse levels as a QSGD-MaxNorm record of b1 bits
+ *     (header [M1, b1, n]) followed by the fine levels as a QSGD-MaxNorm
+ *     record of b2 bits (header [M2, b2, n]);
+ *   - the merge sums each scale's levels over the workers in integers, scales
+ *     each sum once (the QSGD-MaxNorm merge of that scale's records) and adds
+ *     the two: out = A + B.  Both integer sums can be formed by an
+ *     all-reduce, as in the one-scale scheme.
+ * With b1 = 2 (s1 = 1) the two scales coincide, every element with |g| <= M
+ * is fine, and the fine record is the QSGD-MaxNorm record of b2 bits. */
+
+int64_t oracle_qsgd_mnts_words(int64_t n, int b1, int b2)
+{
+    return oracle_qsgd_words(n, b1) + oracle_qsgd_words(n, b2);
+}
+
+/* The fine scale: the coarse scale's quantization step. */
+float oracle_qsgd_mnts_fine_scale(float M, int b1)
+{
+    return M / (float)qsgd_levels(b1);
+}
+
+void oracle_qsgd_mnts_quantize(const float *grad, uint32_t *compr, int64_t n, int b1, int b2,
+                               uint64_t seed, float M)
+{
+    float M2 = oracle_qsgd_mnts_fine_scale(M, b1);
+    uint32_t *coarse = compr;
+    uint32_t *fine = compr + oracle_qsgd_words(n, b1);
+    coarse[0] = bits_of(M);
+    coarse[1] = bits_of((float)b1);
+    coarse[2] = bits_of((float)n);
+    fine[0] = bits_of(M2);
+    fine[1] = bits_of((float)b2);
+    fine[2] = bits_of((float)n);
+    for (int64_t w = 0; w < (n * b1 + 31) / 32; ++w)
+        coarse[3 + w] = 0u;
+    for (int64_t w = 0; w < (n * b2 + 31) / 32; ++w)
+        fine[3 + w] = 0u;
+    for (int64_t e = 0; e < n; ++e) {
+        int is_fine = fabsf(grad[e]) <= M2;
+        int32_t q1 = is_fine ? 0 : oracle_qsgd_level(grad[e], M, b1, seed, e);
+        int32_t q2 = is_fine ? oracle_qsgd_level(grad[e], M2, b2, seed, e) : 0;
+        int per1 = 32 / b1, per2 = 32 / b2;
+        coarse[3 + e / per1] |= ((uint32_t)q1 & ((1u << b1) - 1u)) << (32 - b1 * (int)(e % per1 + 1));
+        fine[3 + e / per2] |= ((uint32_t)q2 & ((1u << b2) - 1u)) << (32 - b2 * (int)(e % per2 + 1));
+    }
+}
+
+void oracle_qsgd_mnts_dequant_accumulate(const uint32_t *const *compr, int W, float *out,
+                                         int64_t n, int b1, int b2)
+{
+    int64_t fine_off = oracle_qsgd_words(n, b1);
+    float step1 = float_of(compr[0][0]) / (float)qsgd_levels(b1);
+    float step2 = float_of(compr[0][fine_off]) / (float)qsgd_levels(b2);
+    for (int64_t e = 0; e < n; ++e) {
+        int32_t sum1 = 0, sum2 = 0;
+        for (int w = 0; w < W; ++w) {
+            sum1 += qsgd_level_at(compr[w], e, b1);
+            sum2 += qsgd_level_at(compr[w] + fine_off, e, b2);
+        }
+        float coarse_part = (float)sum1 * step1;
+        float fine_part = (float)sum2 * step2;
+        out[e] = coarse_part + fine_part;
     }
 }
 

@@ -488,6 +488,123 @@ def pin_qsgd_merge_identity(L):
             assert out[e] == want, (b, e, out[e], want)
 
 
+# ========================================================== QSGD-MN-TS ====
+
+def _mnts_split(compr, n, b1):
+    """The two sub-records of a two-scale record: coarse (b1 bits), fine."""
+    k = 3 + -(-(n * b1) // 32)
+    return compr[:k], compr[k:]
+
+
+def _mnts_levels(sub, n, b):
+    return [d for w in sub[3:].tolist() for d in _qsgd_digits(int(w), b)][:n]
+
+
+def pin_qsgd_mnts_reduces_to_qsgd(L):
+    """With b1 = 2 (s1 = 1) the fine scale equals the coarse one: the fine
+    sub-record is the (pinned) QSGD-MaxNorm record of b2 bits, the coarse one
+    holds only its header, and the merge is the QSGD-MaxNorm merge."""
+    rng = np.random.default_rng(41)
+    for b2 in (2, 4, 8):
+        for n in (0, 1, 33, 257):
+            W = 3
+            gs = [(rng.standard_normal(n) * 2).astype(np.float32) for _ in range(W)]
+            M = oracle.qsgd_mn_max(gs, L) if n else F32(1.0)
+            recs, fines = [], []
+            for w in range(W):
+                ts = oracle.qsgd_mnts_quantize(gs[w], 2, b2, 900 + w, M, L)
+                coarse, fine = _mnts_split(ts, n, 2)
+                assert ts.size == oracle.qsgd_mnts_words(n, 2, b2, L) == coarse.size + fine.size
+                assert np.array_equal(fine, oracle.qsgd_mn_quantize(gs[w], b2, 900 + w, M, L))
+                assert coarse[:3].tolist() == [bits_of_f32(M), bits_of_f32(2.0), bits_of_f32(n)]
+                assert not coarse[3:].any()
+                recs.append(ts)
+                fines.append(fine)
+            got = oracle.qsgd_mnts_dequant_accumulate(recs, n, 2, b2, L)
+            want = oracle.qsgd_mn_dequant_accumulate(fines, n, b2, L)
+            assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+
+
+def pin_qsgd_mnts_scale_assignment(L):
+    """Fine scale = binary32(M / s1) (correctly rounded); an element with
+    |g| <= fine scale has its (pinned) QSGD-MaxNorm level on the fine scale
+    with b2 bits and 0 on the coarse one, any other element the reverse;
+    headers [M, b1, n] and [M2, b2, n]; |levels| <= s per scale."""
+    rng = np.random.default_rng(43)
+    for b1 in (4, 8):
+        s1 = 2 ** (b1 - 1) - 1
+        for b2 in (2, 4, 8):
+            s2 = 2 ** (b2 - 1) - 1
+            n = 301
+            g = (rng.standard_normal(n) * 3).astype(np.float32)
+            g[::37] = 50.0
+            M = F32(np.max(np.abs(g)))
+            M2 = oracle.qsgd_mnts_fine_scale(M, b1, L)
+            assert abs(Fraction(float(M2)) - Fraction(float(M)) / s1) <= half_ulp(M2)
+            g[5], g[6] = M2, -M2                                     # on the boundary: fine
+            g[7] = np.nextafter(M2, F32(np.inf))                     # just above: coarse
+            g[8] = -np.nextafter(M2, F32(0))                         # just below: fine
+            seed = 77 + b1 + b2
+            ts = oracle.qsgd_mnts_quantize(g, b1, b2, seed, M, L)
+            coarse, fine = _mnts_split(ts, n, b1)
+            assert coarse[:3].tolist() == [bits_of_f32(M), bits_of_f32(b1), bits_of_f32(n)]
+            assert fine[:3].tolist() == [bits_of_f32(M2), bits_of_f32(b2), bits_of_f32(n)]
+            q1, q2 = _mnts_levels(coarse, n, b1), _mnts_levels(fine, n, b2)
+            for e in range(n):
+                assert abs(q1[e]) <= s1 and abs(q2[e]) <= s2
+                if abs(g[e]) <= M2:
+                    assert q1[e] == 0 and q2[e] == oracle.qsgd_level(g[e], M2, b2, seed, e, L), (b1, b2, e)
+                else:
+                    assert q2[e] == 0 and q1[e] == oracle.qsgd_level(g[e], M, b1, seed, e, L), (b1, b2, e)
+            assert q2[5] == s2 and q2[6] == -s2 and q1[5] == q1[6] == 0
+            assert q2[7] == 0 and q1[7] >= 1 and q1[8] == 0
+
+
+def pin_qsgd_mnts_unbiased(L):
+    """E[value] = g on both scales: value = q1 M / s1 + q2 M2 / s2 averaged
+    over many independent draws matches g within a few standard errors."""
+    draws = 6000
+    b1, b2 = 4, 4
+    s1, s2 = 7, 7
+    M = F32(7.0)                                   # fine scale M2 = 1
+    for gval in (0.37, -0.9, 1.0, 2.6, -6.1):
+        g = np.full(draws, gval, np.float32)
+        ts = oracle.qsgd_mnts_quantize(g, b1, b2, 55, M, L)
+        coarse, fine = _mnts_split(ts, draws, b1)
+        q1 = np.array(_mnts_levels(coarse, draws, b1))
+        q2 = np.array(_mnts_levels(fine, draws, b2))
+        est = (q1 * (7.0 / s1) + q2 * (1.0 / s2)).mean()
+        step = 1.0 / s2 if abs(gval) <= 1.0 else 7.0 / s1
+        sd = step * 0.5 / np.sqrt(draws)
+        assert abs(est - gval) < 5 * sd + 1e-6, (gval, est)
+
+
+def pin_qsgd_mnts_merge_exact(L):
+    """With power-of-two steps (M = 7/8, b1 = 4: coarse step 1/8, fine
+    scale 1/8, b2 = 2: fine step 1/8) every product and the final add are
+    exact: the merge equals (sum of coarse + fine levels) / 8."""
+    rng = np.random.default_rng(47)
+    n, W = 16 * 9 + 5, 8
+    M = F32(0.875)
+    gs = []
+    for _ in range(W):
+        g = (rng.uniform(-0.875, 0.875, n)).astype(np.float32)
+        g[::5] *= F32(0.1)                         # plenty of fine elements
+        gs.append(g)
+    recs = [oracle.qsgd_mnts_quantize(gs[w], 4, 2, 600 + w, M, L) for w in range(W)]
+    out = oracle.qsgd_mnts_dequant_accumulate(recs, n, 4, 2, L)
+    total = np.zeros(n, np.int64)
+    coarse_seen = fine_seen = False
+    for r in recs:
+        coarse, fine = _mnts_split(r, n, 4)
+        q1, q2 = np.array(_mnts_levels(coarse, n, 4)), np.array(_mnts_levels(fine, n, 2))
+        coarse_seen |= bool(q1.any())
+        fine_seen |= bool(q2.any())
+        total += q1 + q2
+    assert coarse_seen and fine_seen
+    assert np.array_equal(out, (total / 8.0).astype(np.float32))
+
+
 # ======================================================= dense ternary ====
 
 def _ternary_bytes(compr, nbytes):
