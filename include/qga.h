@@ -6,8 +6,9 @@
  *        "Approach", "Two bit quantization", "Format of compressed gradient",
  *        "Operators", "Local kvstore".
  *   [GC] gradient-compression README (vineeths96), "About The Project",
- *        "Results": names QSGDMaxNorm quantization (all-reduce compatible)
- *        without a formula; its definition here is this library's own.
+ *        "Results": names QSGDMaxNorm quantization (all-reduce compatible),
+ *        its two-scale and GlobalRandK variants, without formulas; their
+ *        definitions here are this library's own.
  *   [SC11] Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers: As Easy as
  *        1, 2, 3", SC'11 (Philox4x32-10).
  *
@@ -231,6 +232,43 @@ int qga_qsgd_mn_quantize(const float *grad, uint32_t *compr, int64_t n, int bits
  * the scheme all-reduce compatible ([GC] "About The Project"). */
 int qga_qsgd_mn_dequant_accumulate(const uint32_t *const *compr, int num_workers, float *out,
                                    int64_t n, int bits, cudaStream_t stream);
+
+/* ============================= QSGD-MaxNorm with two scales (QSGD-MN-TS) ==
+ * [GC] "Results" names QSGDMaxNormMultiScale quantization run with two
+ * scales, each run labelled with the bit widths of its two scales, and
+ * [GC] "About The Project" counts it among the all-reduce compatible
+ * schemes; no formula is given.  This library's definition:
+ *   coarse scale M1 = M (the global max |g|, e.g. from qga_qsgd_mn_max) with
+ *     bits_coarse bits, s1 = 2^(bits_coarse-1) - 1 levels;
+ *   fine scale M2 = M1 / s1 (one binary32 division: the coarse grid's first
+ *     step) with bits_fine bits, s2 = 2^(bits_fine-1) - 1 levels;
+ *   an element with |g| <= M2 gets its QSGD-MaxNorm level on the fine scale
+ *     (M2, s2) and level 0 on the coarse one; any other element its level on
+ *     the coarse scale (M1, s1) and 0 on the fine one; both use the element's
+ *     QSGD-MaxNorm draw u(e) of the worker's seed.
+ * Record: the coarse levels as a QSGD-MaxNorm record of bits_coarse bits
+ * (header [M1, bits_coarse, n]) immediately followed by the fine levels as a
+ * QSGD-MaxNorm record of bits_fine bits (header [M2, bits_fine, n]).
+ * With bits_coarse = 2 the scales coincide and the fine part is the
+ * QSGD-MaxNorm record of bits_fine bits. */
+
+/* Words of a two-scale record: qga_qsgd_words(n, bits_coarse) +
+ * qga_qsgd_words(n, bits_fine).  Negative on invalid input. */
+int64_t qga_qsgd_mnts_words(int64_t n, int bits_coarse, int bits_fine);
+
+/* One worker's two-scale record; M1 read from *max_in (device).
+ *   grad   float[n];  compr uint32[qga_qsgd_mnts_words(n, ...)], overwritten
+ *   bits_coarse, bits_fine  2, 4 or 8 each (others: QGA_ERR_UNSUPPORTED) */
+int qga_qsgd_mnts_quantize(const float *grad, uint32_t *compr, int64_t n, int bits_coarse,
+                           int bits_fine, uint64_t seed, const float *max_in, cudaStream_t stream);
+
+/* Merge of W two-scale records: out[e] = A + B (binary32), where
+ *   A = (float)(sum_w coarse level) * (M1 / s1),  B = (float)(sum_w fine
+ *   level) * (M2 / s2), M1 and M2 read from worker 0's two headers.
+ * Both level sums are exact integers (all-reduce compatible).
+ *   out  float[n], overwritten. */
+int qga_qsgd_mnts_dequant_accumulate(const uint32_t *const *compr, int num_workers, float *out,
+                                     int64_t n, int bits_coarse, int bits_fine, cudaStream_t stream);
 
 /* ============================================ GRandK-MaxNorm, b bits ==
  * GlobalRandKMaxNorm compression is named in [GC] "Results" (K = 10000) as

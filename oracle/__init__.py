@@ -86,6 +86,7 @@ def _declare(L):
     L.oracle_qsgd_mnts_fine_scale.restype = f32
     L.oracle_qsgd_mnts_fine_scale.argtypes = [f32, i32]
     L.oracle_qsgd_mnts_quantize.argtypes = [vp, vp, i64, i32, i32, u64, f32]
+    L.oracle_qsgd_mnts_levels.argtypes = [f32, f32, i32, i32, u64, i64, vp]
     L.oracle_qsgd_mnts_dequant_accumulate.argtypes = [vp, i32, vp, i64, i32, i32]
     L.oracle_grandk_mn_max.restype = f32
     L.oracle_grandk_mn_max.argtypes = [vp, i32, i64, vp, i64]
@@ -241,6 +242,14 @@ def qsgd_mnts_words(n: int, b1: int, b2: int, L=None) -> int:
 def qsgd_mnts_fine_scale(M, b1: int, L=None) -> np.float32:
     L = L or lib()
     return np.float32(L.oracle_qsgd_mnts_fine_scale(float(M), b1))
+
+
+def qsgd_mnts_levels(grad: float, M, b1: int, b2: int, seed: int, e: int, L=None):
+    """(coarse level, fine level) of one element at position e."""
+    L = L or lib()
+    q = np.zeros(2, np.int32)
+    L.oracle_qsgd_mnts_levels(float(grad), float(M), b1, b2, seed, e, q.ctypes.data)
+    return int(q[0]), int(q[1])
 
 
 def qsgd_mnts_quantize(grad, b1, b2, seed, M, L=None):

@@ -412,6 +412,17 @@ float oracle_qsgd_mnts_fine_scale(float M, int b1)
     return M / (float)qsgd_levels(b1);
 }
 
+/* The two levels of element e: q[0] on the coarse scale, q[1] on the fine
+ * one (one of them is 0). */
+void oracle_qsgd_mnts_levels(float grad, float M, int b1, int b2, uint64_t seed, int64_t e,
+                             int32_t q[2])
+{
+    float M2 = oracle_qsgd_mnts_fine_scale(M, b1);
+    int is_fine = fabsf(grad) <= M2;
+    q[0] = is_fine ? 0 : oracle_qsgd_level(grad, M, b1, seed, e);
+    q[1] = is_fine ? oracle_qsgd_level(grad, M2, b2, seed, e) : 0;
+}
+
 void oracle_qsgd_mnts_quantize(const float *grad, uint32_t *compr, int64_t n, int b1, int b2,
                                uint64_t seed, float M)
 {
@@ -429,12 +440,11 @@ void oracle_qsgd_mnts_quantize(const float *grad, uint32_t *compr, int64_t n, in
     for (int64_t w = 0; w < (n * b2 + 31) / 32; ++w)
         fine[3 + w] = 0u;
     for (int64_t e = 0; e < n; ++e) {
-        int is_fine = fabsf(grad[e]) <= M2;
-        int32_t q1 = is_fine ? 0 : oracle_qsgd_level(grad[e], M, b1, seed, e);
-        int32_t q2 = is_fine ? oracle_qsgd_level(grad[e], M2, b2, seed, e) : 0;
+        int32_t q[2];
+        oracle_qsgd_mnts_levels(grad[e], M, b1, b2, seed, e, q);
         int per1 = 32 / b1, per2 = 32 / b2;
-        coarse[3 + e / per1] |= ((uint32_t)q1 & ((1u << b1) - 1u)) << (32 - b1 * (int)(e % per1 + 1));
-        fine[3 + e / per2] |= ((uint32_t)q2 & ((1u << b2) - 1u)) << (32 - b2 * (int)(e % per2 + 1));
+        coarse[3 + e / per1] |= ((uint32_t)q[0] & ((1u << b1) - 1u)) << (32 - b1 * (int)(e % per1 + 1));
+        fine[3 + e / per2] |= ((uint32_t)q[1] & ((1u << b2) - 1u)) << (32 - b2 * (int)(e % per2 + 1));
     }
 }
 

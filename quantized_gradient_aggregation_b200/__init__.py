@@ -71,6 +71,9 @@ _SIGS = {
     "qga_qsgd_mn_max": (_i32, [_VPP, _i32, _i64, _vp, _vp]),
     "qga_qsgd_mn_quantize": (_i32, [_vp, _vp, _i64, _i32, _u64, _vp, _vp]),
     "qga_qsgd_mn_dequant_accumulate": (_i32, [_VPP, _i32, _vp, _i64, _i32, _vp]),
+    "qga_qsgd_mnts_words": (_i64, [_i64, _i32, _i32]),
+    "qga_qsgd_mnts_quantize": (_i32, [_vp, _vp, _i64, _i32, _i32, _u64, _vp, _vp]),
+    "qga_qsgd_mnts_dequant_accumulate": (_i32, [_VPP, _i32, _vp, _i64, _i32, _i32, _vp]),
     "qga_grandk_mn_max": (_i32, [_VPP, _i32, _i64, _vp, _i64, _vp, _vp]),
     "qga_grandk_mn_quantize": (_i32, [_vp, _i64, _vp, _i64, _vp, _i32, _u64, _vp, _vp]),
     "qga_grandk_mn_dequant_accumulate": (_i32, [_VPP, _i32, _vp, _i64, _vp, _i64, _i32, _vp]),
@@ -331,6 +334,40 @@ def qga_qsgd_mn_dequant_accumulate(comprs, out, bits, stream=None):
     _check(_lib.qga_qsgd_mn_dequant_accumulate(arr, len(comprs), _ptr(out), n, bits,
                                                _stream(stream, out.device)),
            "qga_qsgd_mn_dequant_accumulate")
+
+
+# ======================================================= QSGD-MN-TS ====
+
+def qga_qsgd_mnts_words(n: int, bits_coarse: int, bits_fine: int) -> int:
+    w = _lib.qga_qsgd_mnts_words(n, bits_coarse, bits_fine)
+    if w < 0:
+        raise QGAError(int(w), "qga_qsgd_mnts_words")
+    return int(w)
+
+
+def qga_qsgd_mnts_quantize(grad, compr, bits_coarse, bits_fine, seed, max_in, stream=None):
+    """Two-scale record of ``grad``: coarse levels on M (``max_in``), fine
+    levels on M / s_coarse; see include/qga.h."""
+    n = grad.numel()
+    _need(grad, torch.float32, None, "grad")
+    _need(compr, torch.int32, qga_qsgd_mnts_words(n, bits_coarse, bits_fine), "compr")
+    _need(max_in, torch.float32, 1, "max_in")
+    _check(_lib.qga_qsgd_mnts_quantize(_ptr(grad), _ptr(compr), n, bits_coarse, bits_fine,
+                                       seed & ((1 << 64) - 1), _ptr(max_in),
+                                       _stream(stream, grad.device)),
+           "qga_qsgd_mnts_quantize")
+
+
+def qga_qsgd_mnts_dequant_accumulate(comprs, out, bits_coarse, bits_fine, stream=None):
+    n = out.numel()
+    _need(out, torch.float32, None, "out")
+    words = qga_qsgd_mnts_words(n, bits_coarse, bits_fine)
+    for i, c in enumerate(comprs):
+        _need(c, torch.int32, words, f"compr[{i}]")
+    arr, keep = _ptr_array(comprs)
+    _check(_lib.qga_qsgd_mnts_dequant_accumulate(arr, len(comprs), _ptr(out), n, bits_coarse,
+                                                 bits_fine, _stream(stream, out.device)),
+           "qga_qsgd_mnts_dequant_accumulate")
 
 
 # ======================================================== GRandK-MN ====

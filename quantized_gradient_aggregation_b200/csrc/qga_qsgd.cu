@@ -174,29 +174,12 @@ __global__ void __launch_bounds__(kThreads)
 }
 
 // ----------------------------------------------------------------- merge ----
-// Integer sum of the W workers' levels, a whole record word at a time.  XOR
-// with the sign bit of every b-bit field turns a two's-complement level q
-// into q + 2^(b-1) in [0, 2^b); masking every fourth (b = 2, 4) or every
-// other (b = 8) field spreads the biased fields into 8-bit (b = 2) or 16-bit
-// lanes of 32-bit registers, where one integer add sums a lane group over a
-// worker without carries crossing lanes (at most 64 workers: 64 * 3 < 2^8,
-// 64 * 255 < 2^16).  At the end each lane's sum, minus W * 2^(b-1), is the
-// exact integer level sum, converted to binary32 exactly through the 2^23
-// magic number (it is below 2^23) and scaled once by fl(M / s).
-//
-// A thread owns whole words: word l of each 32-word block of its warp (for
-// b = 2, also word 32 + l, loaded together for more bytes in flight), and
-// stores its 32/b outputs as 128-bit (b = 8) or 256-bit rows.
-template <int B> struct Swar {
-    static constexpr int kFields = 32 / B;          // elements per word
-    static constexpr int kLaneBits = B == 2 ? 8 : 16;
-    static constexpr int kLanesPerReg = 32 / kLaneBits;
-    static constexpr int kRegs = kFields / kLanesPerReg;
-    static constexpr uint32_t kSign = B == 2 ? 0xAAAAAAAAu : (B == 4 ? 0x88888888u : 0x80808080u);
-    // fields j, j + kRegs, j + 2 kRegs, ... (counted from the least significant) -> register j
-    static constexpr uint32_t kMask = B == 2 ? 0x03030303u : (B == 4 ? 0x000F000Fu : 0x00FF00FFu);
-    static constexpr int kSlots = B == 2 ? 2 : 1;   // words per thread (measured best)
-};
+// Integer sum of the W workers' levels a whole record word at a time (Swar,
+// swar_add_word in qga_qsgd_level.cuh).  A thread owns whole words: word l of
+// each 32-word block of its warp (for b = 2, also word 32 + l, loaded
+// together for more bytes in flight), and stores its 32/b outputs as 128-bit
+// (b = 8) or 256-bit rows.
+template <int B> constexpr int kMergeSlotsFor = B == 2 ? 2 : 1; // words per thread (measured best)
 
 // Outputs of one record word from its lane sums: element e sits in field
 // kFields - 1 - e (counted from the least significant).
@@ -208,12 +191,8 @@ __device__ __forceinline__ void merge_store_word(const uint32_t (&acc)[Swar<B>::
     using S = Swar<B>;
     float v[S::kFields];
 #pragma unroll
-    for (int e = 0; e < S::kFields; ++e) {
-        const int f = S::kFields - 1 - e;
-        const uint32_t sum =
-            (acc[f % S::kRegs] >> (S::kLaneBits * (f / S::kRegs))) & ((1u << S::kLaneBits) - 1u);
-        v[e] = __fmul_rn(__fsub_rn(__uint_as_float(0x4B000000u | sum), offset), step);
-    }
+    for (int e = 0; e < S::kFields; ++e)
+        v[e] = __fmul_rn(__fsub_rn(__uint_as_float(0x4B000000u | swar_field_sum<B>(acc, e)), offset), step);
     const int64_t e0 = kw * S::kFields;
     if (kVec && e0 + S::kFields <= n) {
         if (S::kFields == 4)
@@ -228,16 +207,6 @@ __device__ __forceinline__ void merge_store_word(const uint32_t (&acc)[Swar<B>::
             if (e0 + e < n)
                 st_stream_f1(out + e0 + e, v[e]);
     }
-}
-
-template <int B>
-__device__ __forceinline__ void merge_add_word(uint32_t (&acc)[Swar<B>::kRegs], uint32_t word)
-{
-    using S = Swar<B>;
-    const uint32_t biased = word ^ S::kSign;
-#pragma unroll
-    for (int j = 0; j < S::kRegs; ++j)
-        acc[j] += (biased >> (B * j)) & S::kMask;
 }
 
 template <int B, bool kVec>
@@ -256,7 +225,7 @@ __global__ void __launch_bounds__(kThreads)
     const float offset = 8388608.0f + (float)(W << (B - 1));
     const int64_t nwords = (n * B + 31) >> 5;
     const int64_t stride = (int64_t)gridDim.x * kThreads;
-    if constexpr (S::kSlots == 1) {
+    if constexpr (kMergeSlotsFor<B> == 1) {
         for (int64_t kw = (int64_t)blockIdx.x * kThreads + threadIdx.x; kw < nwords; kw += stride) {
             uint32_t acc[S::kRegs] = {};
             for (int wb = 0; wb < W; wb += kBatch) {
@@ -268,7 +237,7 @@ __global__ void __launch_bounds__(kThreads)
                 for (int i = 0; i < kBatch; ++i) {
                     if (wb + i >= W) // warp-uniform
                         break;
-                    merge_add_word<B>(acc, words[i]);
+                    swar_add_word<B>(acc, words[i]);
                 }
             }
             merge_store_word<B, kVec>(acc, kw, offset, step, out, n);
@@ -293,8 +262,8 @@ __global__ void __launch_bounds__(kThreads)
                 for (int i = 0; i < kBatch; ++i) {
                     if (wb + i >= W) // warp-uniform
                         break;
-                    merge_add_word<B>(acc0, w0[i]);
-                    merge_add_word<B>(acc1, w1[i]);
+                    swar_add_word<B>(acc0, w0[i]);
+                    swar_add_word<B>(acc1, w1[i]);
                 }
             }
             if (k0 < nwords)
@@ -323,7 +292,7 @@ template <int B>
 unsigned merge_grid(int64_t n, int resident)
 {
     const int64_t nwords = (n * B + 31) >> 5;
-    const int64_t per_block = (int64_t)kThreads * Swar<B>::kSlots;
+    const int64_t per_block = (int64_t)kThreads * kMergeSlotsFor<B>;
     return grid_for((nwords + per_block - 1) / per_block, resident, kQsgdMergeWaves<B>);
 }
 

@@ -60,14 +60,14 @@ __device__ __forceinline__ int32_t qsgd_level_exact(float g, float M, float u)
 }
 
 // The same level with one multiply instead of the division, for a finite
-// positive M, and k = fl(s / M).  Only floor(t) matters, so: t' = fl(fl(|g| k)
-// + u) is within 2^-15 of the definition's t whenever t' < s + 1 (each of the
-// two is within 1.9e-5 of the exact real |g| s / M + u: two relative
-// roundings of at most 2^-24 on a value below 128, plus half an ulp below
-// 128), and any t' >= s + 1 caps both to s.  So wherever t' is at least
-// 2^-14 away from an integer, floor(t') == floor(t); otherwise (or if t' is
-// not finite) the exact sequence decides.  Results are identical to
-// qsgd_level_exact for every input.
+// positive M, and k = fl(s / M).  Only floor(t) matters.  Each of t' =
+// fl(fl(|g| k) + u) and the definition's t is within 1.9e-5 of the exact real
+// |g| s / M + u whenever it is below s + 1 (two relative roundings of at most
+// 2^-24 on a value below 128, 1.5e-5, plus half an ulp below 128, 3.8e-6), so
+// |t - t'| <= 3.8e-5, below 2^-14 (6.1e-5); any t' >= s + 1 caps both to s.
+// So wherever t' is at least 2^-14 away from an integer, floor(t') ==
+// floor(t); otherwise (or if t' is not finite) the exact sequence decides.
+// Results are identical to qsgd_level_exact for every input.
 //   x: the draw's output word; u = (x >> 8) 2^-24 enters the sum through one
 //   fused multiply-add, whose product is exact, so the sum is the same single
 //   rounding of |g| k + u as a separate add of u.
@@ -85,6 +85,104 @@ __device__ __forceinline__ int32_t qsgd_level(float g, float M, float k, uint32_
     if (!(fabsf(__fsub_rn(d, 0.5f)) <= 0.5f - kMargin))
         return qsgd_level_exact<B>(g, M, __fmul_rn(m, 0x1p-24f));
     return (int32_t)copysignf(fminf(fl, s), g); // g = -0 gives 0
+}
+
+// ------------------------------------------------ fixed-point fast level --
+// The level of one element without the division and without conversions
+// between integers and floats, for a finite positive M and k = fl(s / M).
+// 2^E must exceed every level count s the caller uses (E = b - 1 for one
+// scale of b bits).  With F = 23 - E fraction bits:
+//   a  = fl(|g| k)                      (one multiply)
+//   X  = fl(a + 2^E)                    bits(X) - bits(2^E) = a rounded to a
+//                                       multiple of 2^-F, as an integer
+//   T  = that integer + (x >> (32 - F)) the draw u truncated to F fraction bits
+//   level = min(floor(T / 2^F), s),  signed by g
+// T / 2^F differs from the definition's t by at most 2^(E-21): a and
+// fl(fl(|g| / M) s) are each within 2^(E-23) of the exact |g| s / M (two
+// relative roundings of 2^-24 on a value below 2^E), a's rounding to the grid
+// adds 2^-(F+1) = 2^(E-24), the truncation of u less than 2^-F = 2^(E-23),
+// and the definition's last rounding 2^(E-24); the sum is below 2^(E-21),
+// 4 units of 2^-F.  So wherever T is at least kFixMargin = 8 units away from
+// a multiple of 2^F, floor(T / 2^F) = floor(t).  Near an integer (fraction
+// of T within 8 units), and for a not below 2^E (X >= 2^(E+1), which also
+// catches an infinite or NaN a), the caller recomputes the level by the
+// definition's operations (qsgd_level_exact).  Levels at or above s need no
+// margin: both sides cap them to s.  The checks are accumulated over a
+// lane's elements (fmin, xmax) so that one test per tile decides.
+//   x: the draw's Philox output word (u = (x >> 8) 2^-24).
+template <int E> struct FixLevel {
+    static constexpr int F = 23 - E;
+    static constexpr uint32_t kOne = (127u + E) << 23;  // binary32 bits of 2^E
+    static constexpr uint32_t kTwo = (128u + E) << 23;  // bits of 2^(E+1)
+    static constexpr uint32_t kMargin = 8;              // units of 2^-F
+    static constexpr uint32_t kFrac = (1u << F) - 1u;
+    // the per-lane accumulators start here; recompute iff needs_exact()
+    static __device__ __forceinline__ void reset(uint32_t &fmin, uint32_t &xmax)
+    {
+        fmin = 0xFFFFFFFFu;
+        xmax = 0u;
+    }
+    static __device__ __forceinline__ bool needs_exact(uint32_t fmin, uint32_t xmax)
+    {
+        return fmin < 2u * kMargin || xmax >= kTwo;
+    }
+};
+
+template <int E>
+__device__ __forceinline__ int32_t qsgd_level_fixed(float g, float k, uint32_t s, uint32_t x,
+                                                    uint32_t &fmin, uint32_t &xmax)
+{
+    using Fx = FixLevel<E>;
+    const float a = __fmul_rn(fabsf(g), k);
+    const uint32_t xb = __float_as_uint(__fadd_rn(a, (float)(1 << E)));
+    // T + kMargin: its floor equals T's wherever the fraction of T + kMargin is
+    // at least 2 kMargin, which is what the accumulated check demands
+    const uint32_t t8 = xb + (x >> (32 - Fx::F)) + (Fx::kMargin - Fx::kOne);
+    fmin = min(fmin, t8 & Fx::kFrac);
+    xmax = max(xmax, xb);
+    const uint32_t level = min(t8 >> Fx::F, s);
+    const uint32_t sg = (uint32_t)((int32_t)__float_as_uint(g) >> 31); // all ones if g < 0
+    return (int32_t)((level ^ sg) - sg);
+}
+
+// ------------------------------------------------- integer sum of levels --
+// The merges add the W workers' levels a whole record word at a time.  XOR
+// with the sign bit of every b-bit field turns a two's-complement level q
+// into q + 2^(b-1) in [0, 2^b); masking every fourth (b = 2, 4) or every
+// other (b = 8) field spreads the biased fields into 8-bit (b = 2) or 16-bit
+// lanes of 32-bit registers, where one integer add sums a lane group over a
+// worker without carries crossing lanes (at most 64 workers: 64 * 3 < 2^8,
+// 64 * 255 < 2^16).  At the end each lane's sum, minus W * 2^(b-1), is the
+// exact integer level sum; it is below 2^23, so adding it to the bits of
+// 2^23 and subtracting 2^23 + W 2^(b-1) in binary32 converts it exactly.
+template <int B> struct Swar {
+    static constexpr int kFields = 32 / B;          // elements per word
+    static constexpr int kLaneBits = B == 2 ? 8 : 16;
+    static constexpr int kLanesPerReg = 32 / kLaneBits;
+    static constexpr int kRegs = kFields / kLanesPerReg;
+    static constexpr uint32_t kSign = B == 2 ? 0xAAAAAAAAu : (B == 4 ? 0x88888888u : 0x80808080u);
+    // fields j, j + kRegs, j + 2 kRegs, ... (counted from the least significant) -> register j
+    static constexpr uint32_t kMask = B == 2 ? 0x03030303u : (B == 4 ? 0x000F000Fu : 0x00FF00FFu);
+};
+
+template <int B>
+__device__ __forceinline__ void swar_add_word(uint32_t (&acc)[Swar<B>::kRegs], uint32_t word)
+{
+    using S = Swar<B>;
+    const uint32_t biased = word ^ S::kSign;
+#pragma unroll
+    for (int j = 0; j < S::kRegs; ++j)
+        acc[j] += (biased >> (B * j)) & S::kMask;
+}
+
+// The biased sum (level sum + W 2^(b-1)) of element e of the word, element
+// 0 being the most significant field.
+template <int B>
+__device__ __forceinline__ uint32_t swar_field_sum(const uint32_t (&acc)[Swar<B>::kRegs], int e)
+{
+    using S = Swar<B>;
+    const int f = S::kFields - 1 - e;
+    return (acc[f % S::kRegs] >> (S::kLaneBits * (f / S::kRegs))) & ((1u << S::kLaneBits) - 1u);
 }
 
 } // namespace qga

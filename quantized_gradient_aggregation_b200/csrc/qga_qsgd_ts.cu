@@ -1,0 +1,350 @@
+// qga_qsgd_ts.cu -- QSGD-MaxNorm with two scales (QSGD-MN-TS): quantize and
+// merge.  The global max is the one-scale max (qga_qsgd_mn_max).
+//
+// The gradient-compression README (vineeths96), "Results", names
+// QSGDMaxNormMultiScale quantization run with two scales, each run labelled
+// with the bit widths of its two scales, and "About The Project" counts it
+// among the all-reduce compatible schemes; no formula is printed.  This
+// library's definition:
+//   coarse scale M1 = M (global max |g|), b1 bits, s1 = 2^(b1-1) - 1 levels;
+//   fine scale   M2 = fl(M1 / s1) (the coarse grid's first step), b2 bits,
+//                s2 = 2^(b2-1) - 1 levels;
+//   an element with |g| <= M2 is quantized on the fine scale, any other on
+//   the coarse one, each by the QSGD-MaxNorm level of that scale (the draw of
+//   the element, Philox4x32-10 as in qga_qsgd.cu); its level on the other
+//   scale is 0;
+//   record = the coarse levels as a QSGD-MaxNorm record of b1 bits (header
+//   [M1, b1, n]) followed by the fine levels as one of b2 bits (header [M2,
+//   b2, n]);
+//   merge: out = fl(fl((sum_w q1) fl(M1 / s1)) + fl((sum_w q2) fl(M2 / s2))),
+//   both level sums exact in integers, so an all-reduce could form them.
+//
+// Quantize: the one-scale kernel's tile geometry (a warp owns 128 groups of
+// 4 elements, lane l groups l, l+32, l+64, l+96; one Philox block per group),
+// the fixed-point level of qga_qsgd_level.cuh with E = max(b1, b2) - 1 and
+// the scale picked per element, and two packed outputs.  Merge: a lane owns
+// 16 consecutive elements, sums each scale's levels over the workers in SIMD
+// lanes of registers (swar_add_word), converts and scales them once and
+// stores its 16 results as two 256-bit rows.
+
+#include <float.h>
+
+#include "qga_common.cuh"
+#include "qga_qsgd_level.cuh"
+
+namespace qga {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarpsPerBlock = kThreads / kWarp;
+constexpr int kGroupsPerLane = 4;
+constexpr int kTileGroups = kWarp * kGroupsPerLane;
+
+struct RecordSet {
+    const uint32_t *rec[QGA_MAX_WORKERS];
+};
+
+__host__ __device__ constexpr int64_t sub_words(int64_t n, int b) { return 3 + (n * b + 31) / 32; }
+
+// Packs the 4 codes of group gi (piece: first element in the top b bits of
+// its 4b bits) into word gi / (8 / b) of a payload; lanes sharing a word
+// combine with xor-shuffles.  All 32 lanes call this together.
+template <int B>
+__device__ __forceinline__ void store_piece(uint32_t *__restrict__ payload, uint32_t piece, int64_t gi,
+                                            int64_t n, int64_t nwords, int lane)
+{
+    const int64_t valid = n - 4 * gi; // codes of elements >= n are zero
+    if (valid < 4)
+        piece = valid <= 0 ? 0u : (piece & ~((1u << (B * (4 - (int)valid))) - 1u));
+    constexpr int LW = Levels<B>::lanes_per_word;
+    uint32_t word = piece << (32 - 4 * B * (1 + (lane % LW)));
+    if (LW >= 2)
+        word |= __shfl_xor_sync(kFullMask, word, 1);
+    if (LW >= 4)
+        word |= __shfl_xor_sync(kFullMask, word, 2);
+    const int64_t wi = gi / LW;
+    if ((lane % LW) == 0 && wi < nwords)
+        st_stream_u32(payload + wi, word);
+}
+
+template <int B1, int B2, bool kVec>
+__global__ void __launch_bounds__(kThreads)
+    qsgd_ts_quantize_kernel(const float *__restrict__ grad, uint32_t *__restrict__ compr, int64_t n,
+                            uint32_t key0, uint32_t key1, const float *__restrict__ max_in)
+{
+    using L1 = Levels<B1>;
+    using L2 = Levels<B2>;
+    constexpr int E = (B1 > B2 ? B1 : B2) - 1;
+    using Fx = FixLevel<E>;
+    const float M1 = *max_in;
+    const float M2 = __fdiv_rn(M1, (float)L1::s);
+    // fast path for a finite positive M1 whose fine scale is positive too
+    const bool fast = M2 > 0.0f && M1 <= FLT_MAX; // uniform over the grid
+    const float k1 = __fdiv_rn((float)L1::s, M1);
+    const float k2 = __fdiv_rn((float)L2::s, M2);
+    uint32_t *coarse = compr;
+    uint32_t *fine = compr + sub_words(n, B1);
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        coarse[0] = bits_from_f32(M1);
+        coarse[1] = bits_from_f32((float)B1);
+        coarse[2] = bits_from_f32(__ll2float_rn(n));
+        fine[0] = bits_from_f32(M2);
+        fine[1] = bits_from_f32((float)B2);
+        fine[2] = bits_from_f32(__ll2float_rn(n));
+    }
+    const int lane = threadIdx.x & (kWarp - 1);
+    const int64_t full_groups = n >> 2;
+    const int64_t groups = (n + 3) >> 2;
+    const int64_t nwords1 = (n * B1 + 31) >> 5, nwords2 = (n * B2 + 31) >> 5;
+    const int64_t tiles = (groups + kTileGroups - 1) / kTileGroups;
+    const int64_t stride = (int64_t)gridDim.x * kWarpsPerBlock;
+    for (int64_t tile = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5); tile < tiles;
+         tile += stride) {
+        const int64_t g0 = tile * kTileGroups;
+        float gv[kGroupsPerLane][4];
+#pragma unroll
+        for (int j = 0; j < kGroupsPerLane; ++j) {
+            const int64_t gi = g0 + j * kWarp + lane;
+            if (kVec && gi < full_groups) {
+                const float4 v = ld_stream_f4(grad + 4 * gi);
+                gv[j][0] = v.x, gv[j][1] = v.y, gv[j][2] = v.z, gv[j][3] = v.w;
+            } else {
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    gv[j][q] = (4 * gi + q < n) ? ld_stream_f1(grad + 4 * gi + q) : 0.0f;
+            }
+        }
+        uint4 draws[kGroupsPerLane];
+#pragma unroll
+        for (int j = 0; j < kGroupsPerLane; ++j) {
+            const int64_t gi = g0 + j * kWarp + lane;
+            draws[j] = philox4x32_10(make_uint4((uint32_t)gi, (uint32_t)((uint64_t)gi >> 32), 0u, 0u),
+                                     key0, key1);
+        }
+        uint32_t p1[kGroupsPerLane], p2[kGroupsPerLane];
+        uint32_t fmin, xmax;
+        Fx::reset(fmin, xmax);
+#pragma unroll
+        for (int j = 0; j < kGroupsPerLane; ++j) {
+            const uint32_t x[4] = {draws[j].x, draws[j].y, draws[j].z, draws[j].w};
+            p1[j] = p2[j] = 0u;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const bool is_fine = fabsf(gv[j][q]) <= M2;
+                const int32_t lv = qsgd_level_fixed<E>(gv[j][q], is_fine ? k2 : k1,
+                                                       is_fine ? (uint32_t)L2::s : (uint32_t)L1::s, x[q],
+                                                       fmin, xmax);
+                p1[j] |= (is_fine ? 0u : ((uint32_t)lv & L1::mask)) << (B1 * (3 - q));
+                p2[j] |= (is_fine ? ((uint32_t)lv & L2::mask) : 0u) << (B2 * (3 - q));
+            }
+        }
+        if (!fast || Fx::needs_exact(fmin, xmax)) {
+            // rare: this lane's elements by the definition's operations
+#pragma unroll
+            for (int j = 0; j < kGroupsPerLane; ++j) {
+                const uint32_t x[4] = {draws[j].x, draws[j].y, draws[j].z, draws[j].w};
+                p1[j] = p2[j] = 0u;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float u = unit_draw(x[q]);
+                    if (fabsf(gv[j][q]) <= M2)
+                        p2[j] |= ((uint32_t)qsgd_level_exact<B2>(gv[j][q], M2, u) & L2::mask) << (B2 * (3 - q));
+                    else
+                        p1[j] |= ((uint32_t)qsgd_level_exact<B1>(gv[j][q], M1, u) & L1::mask) << (B1 * (3 - q));
+                }
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < kGroupsPerLane; ++j) {
+            const int64_t gi = g0 + j * kWarp + lane;
+            store_piece<B1>(coarse + 3, p1[j], gi, n, nwords1, lane);
+            store_piece<B2>(fine + 3, p2[j], gi, n, nwords2, lane);
+        }
+    }
+}
+
+// ----------------------------------------------------------------- merge ----
+constexpr int kSpan = 16; // elements per lane
+
+// The biased level sums of a lane's 16 elements on one scale of b bits:
+// the span's b/2 words of every worker (payload word span * b/2 + i).
+template <int B>
+__device__ __forceinline__ void span_sums(const RecordSet &set, int W, int64_t payload_off, int64_t span,
+                                          int64_t nwords, uint32_t (&sum)[kSpan])
+{
+    using S = Swar<B>;
+    constexpr int kWordsPerSpan = kSpan * B / 32;
+    uint32_t acc[kWordsPerSpan][S::kRegs] = {};
+    constexpr int kBatch = 4;
+    for (int wb = 0; wb < W; wb += kBatch) {
+        uint32_t words[kBatch][kWordsPerSpan];
+#pragma unroll
+        for (int i = 0; i < kBatch; ++i)
+#pragma unroll
+            for (int c = 0; c < kWordsPerSpan; ++c) {
+                const int64_t k = span * kWordsPerSpan + c;
+                words[i][c] = (wb + i < W && k < nwords) ? ld_stream_u32(set.rec[wb + i] + payload_off + k)
+                                                         : Swar<B>::kSign; // biased 0 of an absent worker
+            }
+#pragma unroll
+        for (int i = 0; i < kBatch; ++i) {
+            if (wb + i >= W) // warp-uniform
+                break;
+#pragma unroll
+            for (int c = 0; c < kWordsPerSpan; ++c)
+                swar_add_word<B>(acc[c], words[i][c]);
+        }
+    }
+#pragma unroll
+    for (int c = 0; c < kWordsPerSpan; ++c)
+#pragma unroll
+        for (int e = 0; e < S::kFields; ++e)
+            sum[c * S::kFields + e] = swar_field_sum<B>(acc[c], e);
+}
+
+template <int B1, int B2, bool kVec>
+__global__ void __launch_bounds__(kThreads)
+    qsgd_ts_merge_kernel(const __grid_constant__ RecordSet set, int W, float *__restrict__ out, int64_t n)
+{
+    const int64_t off2 = sub_words(n, B1) + 3; // payload of the fine sub-record
+    const float step1 = __fdiv_rn(f32_from_bits(set.rec[0][0]), (float)Levels<B1>::s);
+    const float step2 = __fdiv_rn(f32_from_bits(set.rec[0][off2 - 3]), (float)Levels<B2>::s);
+    // 2^23 + W 2^(b-1): the exact conversion's offset and the bias
+    const float bias1 = 8388608.0f + (float)(W << (B1 - 1));
+    const float bias2 = 8388608.0f + (float)(W << (B2 - 1));
+    const int64_t nwords1 = (n * B1 + 31) >> 5, nwords2 = (n * B2 + 31) >> 5;
+    const int64_t spans = (n + kSpan - 1) / kSpan;
+    for (int64_t sp = (int64_t)blockIdx.x * kThreads + threadIdx.x; sp < spans;
+         sp += (int64_t)gridDim.x * kThreads) {
+        uint32_t s1[kSpan], s2[kSpan];
+        span_sums<B1>(set, W, 3, sp, nwords1, s1);
+        span_sums<B2>(set, W, off2, sp, nwords2, s2);
+        float v[kSpan];
+#pragma unroll
+        for (int e = 0; e < kSpan; ++e) {
+            const float a = __fmul_rn(__fsub_rn(__uint_as_float(0x4B000000u | s1[e]), bias1), step1);
+            const float b = __fmul_rn(__fsub_rn(__uint_as_float(0x4B000000u | s2[e]), bias2), step2);
+            v[e] = __fadd_rn(a, b);
+        }
+        const int64_t e0 = sp * kSpan;
+        if (kVec && e0 + kSpan <= n) {
+            st_stream_f8(out + e0, v);
+            st_stream_f8(out + e0 + 8, v + 8);
+        } else {
+#pragma unroll
+            for (int e = 0; e < kSpan; ++e)
+                if (e0 + e < n)
+                    st_stream_f1(out + e0 + e, v[e]);
+        }
+    }
+}
+
+int bits_slot(int bits) { return bits == 2 ? 0 : (bits == 4 ? 1 : (bits == 8 ? 2 : -1)); }
+
+std::atomic<int> occ_tq[3][3][2][64];
+std::atomic<int> occ_tm[3][3][2][64];
+
+constexpr int kTsQuantizeWaves = 8, kTsMergeWaves = 8;
+
+template <int B1, int B2>
+void launch_quantize(const float *grad, uint32_t *compr, int64_t n, uint64_t seed, const float *M,
+                     cudaStream_t stream)
+{
+    const uint32_t k0 = (uint32_t)seed, k1 = (uint32_t)(seed >> 32);
+    const int64_t groups = (n + 3) >> 2;
+    const int64_t tiles = (groups + kTileGroups - 1) / kTileGroups;
+    const int64_t blocks = (tiles + kWarpsPerBlock - 1) / kWarpsPerBlock;
+    auto &occ = occ_tq[bits_slot(B1)][bits_slot(B2)];
+    if (aligned(grad, 16)) {
+        auto k = qsgd_ts_quantize_kernel<B1, B2, true>;
+        k<<<grid_for(blocks, resident_blocks(k, kThreads, occ[0]), kTsQuantizeWaves), kThreads, 0,
+            stream>>>(grad, compr, n, k0, k1, M);
+    } else {
+        auto k = qsgd_ts_quantize_kernel<B1, B2, false>;
+        k<<<grid_for(blocks, resident_blocks(k, kThreads, occ[1]), kTsQuantizeWaves), kThreads, 0,
+            stream>>>(grad, compr, n, k0, k1, M);
+    }
+}
+
+template <int B1, int B2>
+void launch_merge(const RecordSet &set, int W, float *out, int64_t n, cudaStream_t stream)
+{
+    const int64_t spans = (n + kSpan - 1) / kSpan;
+    const int64_t blocks = (spans + kThreads - 1) / kThreads;
+    auto &occ = occ_tm[bits_slot(B1)][bits_slot(B2)];
+    if (aligned(out, 32)) {
+        auto k = qsgd_ts_merge_kernel<B1, B2, true>;
+        k<<<grid_for(blocks, resident_blocks(k, kThreads, occ[0]), kTsMergeWaves), kThreads, 0,
+            stream>>>(set, W, out, n);
+    } else {
+        auto k = qsgd_ts_merge_kernel<B1, B2, false>;
+        k<<<grid_for(blocks, resident_blocks(k, kThreads, occ[1]), kTsMergeWaves), kThreads, 0,
+            stream>>>(set, W, out, n);
+    }
+}
+
+// The (b1, b2) pair as template arguments (every width 2, 4 or 8; checked
+// by the caller).
+#define QGA_TS_DISPATCH(b1, b2, CALL)                                                      \
+    do {                                                                                   \
+        const int p_ = (b1) * 16 + (b2);                                                   \
+        if (p_ == 0x22) { constexpr int B1 = 2, B2 = 2; CALL; }                            \
+        else if (p_ == 0x24) { constexpr int B1 = 2, B2 = 4; CALL; }                       \
+        else if (p_ == 0x28) { constexpr int B1 = 2, B2 = 8; CALL; }                       \
+        else if (p_ == 0x42) { constexpr int B1 = 4, B2 = 2; CALL; }                       \
+        else if (p_ == 0x44) { constexpr int B1 = 4, B2 = 4; CALL; }                       \
+        else if (p_ == 0x48) { constexpr int B1 = 4, B2 = 8; CALL; }                       \
+        else if (p_ == 0x82) { constexpr int B1 = 8, B2 = 2; CALL; }                       \
+        else if (p_ == 0x84) { constexpr int B1 = 8, B2 = 4; CALL; }                       \
+        else { constexpr int B1 = 8, B2 = 8; CALL; }                                       \
+    } while (0)
+
+} // namespace
+} // namespace qga
+
+using namespace qga;
+
+extern "C" int64_t qga_qsgd_mnts_words(int64_t n, int bits_coarse, int bits_fine)
+{
+    if (n < 0)
+        return QGA_ERR_INVALID_ARG;
+    if (bits_slot(bits_coarse) < 0 || bits_slot(bits_fine) < 0)
+        return QGA_ERR_UNSUPPORTED;
+    return sub_words(n, bits_coarse) + sub_words(n, bits_fine);
+}
+
+extern "C" int qga_qsgd_mnts_quantize(const float *grad, uint32_t *compr, int64_t n, int bits_coarse,
+                                      int bits_fine, uint64_t seed, const float *max_in,
+                                      cudaStream_t stream)
+{
+    if (n < 0 || compr == nullptr || !aligned(compr, 4) || max_in == nullptr || !aligned(max_in, 4))
+        return QGA_ERR_INVALID_ARG;
+    if (n > 0 && (grad == nullptr || !aligned(grad, 4)))
+        return QGA_ERR_INVALID_ARG;
+    if (bits_slot(bits_coarse) < 0 || bits_slot(bits_fine) < 0)
+        return QGA_ERR_UNSUPPORTED;
+    QGA_TS_DISPATCH(bits_coarse, bits_fine, (launch_quantize<B1, B2>(grad, compr, n, seed, max_in, stream)));
+    return launch_status();
+}
+
+extern "C" int qga_qsgd_mnts_dequant_accumulate(const uint32_t *const *compr, int num_workers, float *out,
+                                                int64_t n, int bits_coarse, int bits_fine,
+                                                cudaStream_t stream)
+{
+    if (compr == nullptr || num_workers < 1 || num_workers > QGA_MAX_WORKERS || n < 0)
+        return QGA_ERR_INVALID_ARG;
+    if (bits_slot(bits_coarse) < 0 || bits_slot(bits_fine) < 0)
+        return QGA_ERR_UNSUPPORTED;
+    RecordSet set{};
+    for (int w = 0; w < num_workers; ++w) {
+        if (compr[w] == nullptr || !aligned(compr[w], 4))
+            return QGA_ERR_INVALID_ARG;
+        set.rec[w] = compr[w];
+    }
+    if (n == 0)
+        return QGA_OK;
+    if (out == nullptr || !aligned(out, 4))
+        return QGA_ERR_INVALID_ARG;
+    QGA_TS_DISPATCH(bits_coarse, bits_fine, (launch_merge<B1, B2>(set, num_workers, out, n, stream)));
+    return launch_status();
+}

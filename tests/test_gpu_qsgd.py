@@ -202,8 +202,12 @@ def test_quantize_levels_next_to_integer_boundaries(b):
     seed = 987654321
     n = 4096
     rng = np.random.default_rng(b)
-    deltas = np.array([1e-7, -1e-7, 3e-6, -3e-6, 2e-5, -2e-5, 4e-5, -4e-5, 6e-5, -6e-5, 1e-4, -2e-4,
-                       1.3e-4, -1.3e-4, 1.5e-4, -1.5e-4, 3e-4, -3e-4])
+    # The fast level differs from the definition's t by at most 3.8e-5 and
+    # defers to the definition within 2^-14 = 6.1e-5 of an integer: distances
+    # below, inside and above that band, and on both sides of the margin.
+    deltas = np.array([1e-7, -1e-7, 3e-6, -3e-6, 2e-5, -2e-5, 3.7e-5, -3.7e-5, 3.9e-5, -3.9e-5,
+                       4.5e-5, -4.5e-5, 5.5e-5, -5.5e-5, 6.0e-5, -6.0e-5, 6.2e-5, -6.2e-5, 7e-5, -7e-5,
+                       1e-4, -2e-4, 1.3e-4, -1.3e-4, 3e-4, -3e-4])
     g = np.empty(n, np.float32)
     for e in range(n):
         u = oracle.qsgd_uniform(seed, e)

@@ -77,17 +77,17 @@ MUTANTS = [
     ("ternary least significant first", "    for (int64_t k = e % 5; k < 4; ++k)\n        value /= 3;",
      "    for (int64_t k = 0; k < e % 5; ++k)\n        value /= 3;"),
     ("ternary words per 16", "    return 3 + (n + 19) / 20;", "    return 3 + (n + 15) / 16;"),
-    ("ts boundary strict", "int is_fine = fabsf(grad[e]) <= M2;", "int is_fine = fabsf(grad[e]) < M2;"),
+    ("ts boundary strict", "int is_fine = fabsf(grad) <= M2;", "int is_fine = fabsf(grad) < M2;"),
     ("ts fine scale is M", "return M / (float)qsgd_levels(b1);", "return M;"),
-    ("ts fine level with coarse bits", "oracle_qsgd_level(grad[e], M2, b2, seed, e)",
-     "oracle_qsgd_level(grad[e], M2, b1, seed, e)"),
-    ("ts fine draw of the next element", "oracle_qsgd_level(grad[e], M2, b2, seed, e)",
-     "oracle_qsgd_level(grad[e], M2, b2, seed, e + 1)"),
+    ("ts fine level with coarse bits", "oracle_qsgd_level(grad, M2, b2, seed, e)",
+     "oracle_qsgd_level(grad, M2, b1, seed, e)"),
+    ("ts fine draw of the next element", "oracle_qsgd_level(grad, M2, b2, seed, e)",
+     "oracle_qsgd_level(grad, M2, b2, seed, e + 1)"),
     ("ts merge fine step from coarse header", "float step2 = float_of(compr[0][fine_off])",
      "float step2 = float_of(compr[0][0])"),
     ("ts merge drops coarse part", "out[e] = coarse_part + fine_part;", "out[e] = fine_part;"),
-    ("ts fields swapped", "int32_t q1 = is_fine ? 0 : oracle_qsgd_level",
-     "int32_t q1 = !is_fine ? 0 : oracle_qsgd_level"),
+    ("ts fields swapped", "q[0] = is_fine ? 0 : oracle_qsgd_level",
+     "q[0] = !is_fine ? 0 : oracle_qsgd_level"),
     ("grandk draw keyed on coordinate", "q = oracle_qsgd_level(grad[index[k]], M, b, seed, k);",
      "q = oracle_qsgd_level(grad[index[k]], M, b, seed, index[k]);"),
     ("grandk level of position k", "q = oracle_qsgd_level(grad[index[k]], M, b, seed, k);",
