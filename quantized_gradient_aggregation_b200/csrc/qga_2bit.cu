@@ -122,9 +122,35 @@ __global__ void __launch_bounds__(kThreads, QGA_MERGE_MIN_BLOCKS)
     }
 }
 
+// W <= 8: the merge through the table of all 3^W sums (build_sum_table,
+// merge_2bit_table_slice): one table index and one shared-memory load per
+// element instead of W decodes and adds.  The table (26 KB at W = 8) and the
+// per-warp 2 KB output stage fit 5 blocks per SM.
+template <bool kVec, int kW>
+__global__ void __launch_bounds__(kThreads)
+    merge_2bit_table_kernel(const __grid_constant__ RecordSet set, float *__restrict__ out, int64_t n)
+{
+    __shared__ float s_neg[kW], s_pos[kW];
+    __shared__ float s_sum[Pow3<kW>::value];
+    __shared__ float4 s_stage[kWarpsPerBlock][kWarp * 4];
+    if (threadIdx.x < kW) {
+        const uint32_t *r = set.rec[threadIdx.x];
+        s_neg[threadIdx.x] = f32_from_bits(r[0]);
+        s_pos[threadIdx.x] = f32_from_bits(r[1]);
+    }
+    __syncthreads();
+    build_sum_table<kW>(s_sum, [&](int w) { return s_neg[w]; }, [&](int w) { return s_pos[w]; });
+    const int lane = threadIdx.x & (kWarp - 1);
+    const int64_t slices = (n + kTableSliceElems - 1) / kTableSliceElems;
+    for (int64_t sl = first_tile(); sl < slices; sl += tile_stride())
+        merge_2bit_table_slice<kVec, kW, kTableSlots>([&](int w) { return set.rec[w] + 3; }, s_sum, out,
+                                                       n, sl, lane, s_stage[threadIdx.x >> 5]);
+}
+
 std::atomic<int> occ_q_f32_w[64], occ_q_f32_v[64], occ_q_f32_s[64], occ_q_bf16_v[64], occ_q_bf16_s[64];
 std::atomic<int> occ_dq_v[64], occ_dq_s[64];
-std::atomic<int> occ_acc[2][9][64]; // [vec][kW][device]
+std::atomic<int> occ_acc[2][64];    // [vec][device]: W > 8
+std::atomic<int> occ_tab[2][9][64]; // [vec][kW][device]: W <= 8
 
 // Grid waves (see grid_for), measured at n = 138M: quantize in group tiles
 // 270-286 / 263 / 259 / 256 / 258 us at 1 / 8 / 16 / 32 / 128 waves, in
@@ -132,6 +158,10 @@ std::atomic<int> occ_acc[2][9][64]; // [vec][kW][device]
 // 256); dequantize 109 / 97 / 96 / 101 us at 1 / 8 / 16 / 32; merge (W = 8)
 // 180 / 174 / 176 / 181 us at 1 / 8 / 16 / 32.
 constexpr int kQuantizeWaves = 32, kDequantizeWaves = 16, kMergeWaves = 8;
+#ifndef QGA_TABLE_MERGE_WAVES
+#define QGA_TABLE_MERGE_WAVES 1
+#endif
+constexpr int kTableMergeWaves = QGA_TABLE_MERGE_WAVES;
 
 unsigned tiles_grid(int64_t n, int resident, int64_t elems_per_warp, int waves)
 {
@@ -142,10 +172,16 @@ unsigned tiles_grid(int64_t n, int resident, int64_t elems_per_warp, int waves)
 template <bool kVec, int kW>
 void launch_merge_k(const RecordSet &set, int W, float *out, int64_t n, cudaStream_t stream)
 {
-    auto k = dequant_accumulate_2bit_kernel<kVec, kW>;
-    k<<<tiles_grid(n, resident_blocks(k, kThreads, occ_acc[kVec][kW]), kSliceElems, kMergeWaves),
-        kThreads, 0,
-        stream>>>(set, W, out, n);
+    if constexpr (kW > 0) {
+        auto k = merge_2bit_table_kernel<kVec, kW>;
+        k<<<tiles_grid(n, resident_blocks(k, kThreads, occ_tab[kVec][kW]), kTableSliceElems,
+                       kTableMergeWaves),
+            kThreads, 0, stream>>>(set, out, n);
+    } else {
+        auto k = dequant_accumulate_2bit_kernel<kVec, 0>;
+        k<<<tiles_grid(n, resident_blocks(k, kThreads, occ_acc[kVec]), kSliceElems, kMergeWaves),
+            kThreads, 0, stream>>>(set, W, out, n);
+    }
 }
 
 template <bool kVec>

@@ -411,4 +411,204 @@ __device__ __forceinline__ void dequant_accumulate_2bit_slice(int W_runtime, Pay
     __syncwarp();
 }
 
+// ------------------------------------------------------ merge by sum table --
+// With at most 8 workers the merged value of an element depends on nothing
+// but its W codes, and a code reads as one of three values (11 reads as 00).
+// So every sum the merge can produce is an entry of a table of 3^W floats
+// (6561 at W = 8, 26 KB of shared memory): entry i = sum_k d_k 3^k, digit
+// d_k = 0 / 1 / 2 for codes 00 / 01 / 10 of worker k, holds the sum of those
+// codes' values.  The table is filled with the same binary32 adds in worker
+// order as the definition:
+//   T[0] = +0;  for k = 0 .. W-1, i < 3^k:  T[i + 3^k] = T[i] + pos_k,
+//                                            T[i + 2 3^k] = T[i] + neg_k
+// (T[i] for i < 3^k already holds the sum of workers 0 .. k-1 with the later
+// workers' codes 00, and adding their +0 changes nothing: the running sum
+// starts at +0 and is never -0 in round-to-nearest).  Each entry is thus the
+// definition's sum bit for bit, per-worker thresholds included.
+//
+// Per element the merge computes its table index from the W codes and loads
+// one float: the W sequential adds and decodes per element leave the loop.
+// The index is formed for the 16 elements of a word position at once, in
+// fields of wider and wider registers (SIMD within a register):
+//   - every code 11 is cleared to 00;
+//   - even and odd 2-bit fields go to the low half of 4-bit nibbles;
+//   - two workers combine in a nibble as d_k + 3 d_{k+1} (at most 8);
+//   - two such pairs combine in a byte (at most 80: workers 0-3, and 4-7);
+//   - the two groups combine in 16-bit halves as 4 (A + 81 B), the table
+//     offset in bytes (at most 26240).
+// Integer adds of fields never carry into the neighbouring field: every field
+// is wide enough for its largest value.
+template <int W> struct Pow3 {
+    static constexpr int value = 3 * Pow3<W - 1>::value;
+};
+template <> struct Pow3<0> {
+    static constexpr int value = 1;
+};
+constexpr int kTableMaxWorkers = 8;
+
+// Fill T (3^kW floats of shared memory) from the workers' thresholds.  All
+// threads of the block take part; ends with a barrier.
+template <int kW, typename NegOf, typename PosOf>
+__device__ __forceinline__ void build_sum_table(float *T, NegOf neg_of, PosOf pos_of)
+{
+    if (threadIdx.x == 0)
+        T[0] = 0.0f;
+    __syncthreads();
+    int P = 1;
+#pragma unroll
+    for (int k = 0; k < kW; ++k) {
+        const float pos = pos_of(k), neg = neg_of(k);
+        for (int i = threadIdx.x; i < 2 * P; i += blockDim.x) {
+            const bool one = i < P;
+            const int j = one ? i : i - P;
+            T[j + (one ? P : 2 * P)] = __fadd_rn(T[j], one ? pos : neg);
+        }
+        __syncthreads();
+        P *= 3;
+    }
+}
+
+// A record word with every code 11 turned into 00.
+__device__ __forceinline__ uint32_t clear_code_11(uint32_t w)
+{
+    const uint32_t t = w & (w >> 1) & 0x55555555u; // low bit of each 11
+    return w ^ (t * 3u);
+}
+
+// Byte offsets into the sum table of the 16 elements of one word position:
+// wd[k] is worker k's word (k < kW), off[p] the offset of element p (element
+// p's code sits in bits 31-2p .. 30-2p).
+template <int kW>
+__device__ __forceinline__ void sum_table_offsets(const uint32_t (&wd)[kTableMaxWorkers],
+                                                  uint32_t (&off)[16])
+{
+    static_assert(kW >= 1 && kW <= kTableMaxWorkers, "table merge: 1..8 workers");
+    // nibble i of e[k] / o[k] = field 2i / 2i+1 of worker k (field q = bits 2q..2q+1)
+    uint32_t e[kTableMaxWorkers], o[kTableMaxWorkers];
+#pragma unroll
+    for (int k = 0; k < kW; ++k) {
+        const uint32_t c = clear_code_11(wd[k]);
+        e[k] = c & 0x33333333u;
+        o[k] = (c >> 2) & 0x33333333u;
+    }
+    // pairs of workers: d_2j + 3 d_2j+1 per nibble
+    constexpr int kPairs = (kW + 1) / 2;
+    uint32_t pe[4], po[4];
+#pragma unroll
+    for (int j = 0; j < kPairs; ++j) {
+        pe[j] = e[2 * j];
+        po[j] = o[2 * j];
+        if (2 * j + 1 < kW) {
+            pe[j] += 3u * e[2 * j + 1];
+            po[j] += 3u * o[2 * j + 1];
+        }
+    }
+    // groups of two pairs, in byte lanes; X = 0..3 holds the fields
+    // 4b + {0, 2, 1, 3}[X] in byte b
+    constexpr int kGroups = (kPairs + 1) / 2;
+    uint32_t g[2][4];
+#pragma unroll
+    for (int h = 0; h < kGroups; ++h) {
+        const uint32_t lo_e = pe[2 * h] & 0x0F0F0F0Fu, hi_e = (pe[2 * h] >> 4) & 0x0F0F0F0Fu;
+        const uint32_t lo_o = po[2 * h] & 0x0F0F0F0Fu, hi_o = (po[2 * h] >> 4) & 0x0F0F0F0Fu;
+        g[h][0] = lo_e;
+        g[h][1] = hi_e;
+        g[h][2] = lo_o;
+        g[h][3] = hi_o;
+        if (2 * h + 1 < kPairs) {
+            g[h][0] += 9u * (pe[2 * h + 1] & 0x0F0F0F0Fu);
+            g[h][1] += 9u * ((pe[2 * h + 1] >> 4) & 0x0F0F0F0Fu);
+            g[h][2] += 9u * (po[2 * h + 1] & 0x0F0F0F0Fu);
+            g[h][3] += 9u * ((po[2 * h + 1] >> 4) & 0x0F0F0F0Fu);
+        }
+    }
+    constexpr int kBase[4] = {0, 2, 1, 3};
+#pragma unroll
+    for (int X = 0; X < 4; ++X) {
+        // 16-bit halves: `ev` holds bytes 0 and 2 of the groups, `od` bytes 1 and 3
+        uint32_t ev = 4u * (g[0][X] & 0x00FF00FFu);
+        uint32_t od = 4u * ((g[0][X] >> 8) & 0x00FF00FFu);
+        if (kGroups > 1) {
+            ev += 324u * (g[1][X] & 0x00FF00FFu);
+            od += 324u * ((g[1][X] >> 8) & 0x00FF00FFu);
+        }
+        const int q = kBase[X]; // field of byte 0; element p = 15 - field
+        off[15 - q] = ev & 0xFFFFu;
+        off[15 - (q + 8)] = ev >> 16;
+        off[15 - (q + 4)] = od & 0xFFFFu;
+        off[15 - (q + 12)] = od >> 16;
+    }
+}
+
+// Words per lane of a table-merge slice (build-time setting; the default is
+// the measured best).
+#ifndef QGA_TABLE_MERGE_SLOTS
+#define QGA_TABLE_MERGE_SLOTS 2
+#endif
+constexpr int kTableSlots = QGA_TABLE_MERGE_SLOTS;
+constexpr int64_t kTableSliceElems = (int64_t)kWarp * kTableSlots * 16;
+
+// Merge slice `slice` of kW <= 8 records through the sum table T (built by
+// build_sum_table for the same records).  A warp's slice is 32 kS consecutive
+// words; lane l owns words l, 32 + l, ..., loads all of its words of every
+// worker before using any (merge_2bit_table_load), and computes the 16 sums
+// of each (merge_2bit_table_store).  The sums leave through `stage` (this
+// warp's 2 KB, 128 float4) one word slot at a time, as fully coalesced
+// 128-bit rows (xor-swizzled: both sides free of bank conflicts).  All 32
+// lanes must call these together (warp-uniform `slice`).
+// skip: a worker whose words the caller fills in itself (-1: none).
+template <int kW, int kS, typename PayloadOf>
+__device__ __forceinline__ void merge_2bit_table_load(PayloadOf payload_of, int64_t nwords, int64_t slice,
+                                                      int lane, int skip,
+                                                      uint32_t (&wd)[kS][kTableMaxWorkers])
+{
+#pragma unroll
+    for (int s = 0; s < kS; ++s) {
+        const int64_t k = (slice * kS + s) * kWarp + lane;
+#pragma unroll
+        for (int w = 0; w < kTableMaxWorkers; ++w)
+            wd[s][w] = (w < kW && w != skip && k < nwords) ? ld_stream_u32(payload_of(w) + k) : 0u;
+    }
+}
+
+template <bool kVec, int kW, int kS>
+__device__ __forceinline__ void merge_2bit_table_store(const uint32_t (&wd)[kS][kTableMaxWorkers],
+                                                       const float *T, float *__restrict__ out, int64_t n,
+                                                       int64_t slice, int lane, float4 *__restrict__ stage)
+{
+    const char *tb = reinterpret_cast<const char *>(T);
+    const int f = (lane >> 1) & 3;
+#pragma unroll
+    for (int s = 0; s < kS; ++s) {
+        uint32_t off[16];
+        sum_table_offsets<kW>(wd[s], off);
+        float v[16];
+#pragma unroll
+        for (int p = 0; p < 16; ++p)
+            v[p] = *reinterpret_cast<const float *>(tb + off[p]);
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+            stage[lane * 4 + (c ^ f)] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+        __syncwarp();
+        const int64_t g0 = (slice * kS + s) * kWarp * 4; // first group of this word slot
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int q = j * kWarp + lane;
+            store_group<kVec>(out, n, g0 + q, stage[stage_slot(q >> 2, q & 3)]);
+        }
+        __syncwarp();
+    }
+}
+
+template <bool kVec, int kW, int kS, typename PayloadOf>
+__device__ __forceinline__ void merge_2bit_table_slice(PayloadOf payload_of, const float *T,
+                                                       float *__restrict__ out, int64_t n,
+                                                       int64_t slice, int lane,
+                                                       float4 *__restrict__ stage)
+{
+    uint32_t wd[kS][kTableMaxWorkers];
+    merge_2bit_table_load<kW, kS>(payload_of, (n + 15) >> 4, slice, lane, -1, wd);
+    merge_2bit_table_store<kVec, kW, kS>(wd, T, out, n, slice, lane, stage);
+}
+
 } // namespace qga

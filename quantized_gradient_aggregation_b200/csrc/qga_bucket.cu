@@ -153,19 +153,76 @@ __global__ void __launch_bounds__(kThreads, 3)
     }
 }
 
+// W <= 8: each chunk's tensor merged through the table of its 3^W sums
+// (build_sum_table, merge_2bit_table_slice); the table is rebuilt only when
+// the block moves on to a chunk of another tensor.
+template <int kW>
+__global__ void __launch_bounds__(kThreads)
+    merge_2bit_table_bucket_kernel(const __grid_constant__ MergeTable tab, float *__restrict__ out)
+{
+    __shared__ const uint32_t *s_payload[kW];
+    __shared__ float s_neg[kW], s_pos[kW];
+    __shared__ float s_sum[Pow3<kW>::value];
+    __shared__ float4 s_stage[kWarpsPerBlock][kWarp * 4];
+    static_assert(kMergeChunkElems % kTableSliceElems == 0, "whole slices per chunk");
+    constexpr int64_t kChunkSlices = kMergeChunkElems / kTableSliceElems;
+    const int lane = threadIdx.x & (kWarp - 1);
+    const int warp = threadIdx.x >> 5;
+    int loaded = -1; // the row whose table is in shared memory (block-uniform)
+    for (int64_t chunk = blockIdx.x; chunk < tab.total_chunks; chunk += gridDim.x) {
+        const int t = owner_row(tab, chunk);
+        const MergeRow &row = tab.row[t];
+        if (t != loaded) {
+            __syncthreads(); // the previous tensor's readers of s_* are done
+            if (threadIdx.x < kW) {
+                const uint32_t *rec = tab.bucket[threadIdx.x] + row.word_off;
+                s_payload[threadIdx.x] = rec + 3;
+                s_neg[threadIdx.x] = f32_from_bits(rec[0]);
+                s_pos[threadIdx.x] = f32_from_bits(rec[1]);
+            }
+            __syncthreads();
+            build_sum_table<kW>(s_sum, [&](int w) { return s_neg[w]; }, [&](int w) { return s_pos[w]; });
+            loaded = t;
+        }
+        const int64_t c = chunk - row.chunk_begin;
+        const int64_t slices = (row.n + kTableSliceElems - 1) / kTableSliceElems;
+        const int64_t s_end = min((c + 1) * kChunkSlices, slices);
+        float *o = out + row.elem_off;
+        auto payload_of = [&](int w) { return s_payload[w]; };
+        if (row.vec) {
+            for (int64_t sl = c * kChunkSlices + warp; sl < s_end; sl += kWarpsPerBlock)
+                merge_2bit_table_slice<true, kW, kTableSlots>(payload_of, s_sum, o, row.n, sl, lane,
+                                                              s_stage[warp]);
+        } else {
+            for (int64_t sl = c * kChunkSlices + warp; sl < s_end; sl += kWarpsPerBlock)
+                merge_2bit_table_slice<false, kW, kTableSlots>(payload_of, s_sum, o, row.n, sl, lane,
+                                                               s_stage[warp]);
+        }
+    }
+}
+
 std::atomic<int> occ_qb_f32[2][64], occ_qb_bf16[2][64], occ_ab[9][64];
 
 // Grid waves (see grid_for), measured on the BERT-Base bucket: bf16 quantize
 // 186 / 175 / 171 / 173 us at 1 / 8 / 16 / 32 waves; 4-worker merge 113 /
 // 109 / 109 us at 1 / 8 / 16.
-constexpr int kBucketQuantizeWaves = 16, kBucketMergeWaves = 8;
+#ifndef QGA_BUCKET_MERGE_WAVES
+#define QGA_BUCKET_MERGE_WAVES 8
+#endif
+constexpr int kBucketQuantizeWaves = 16, kBucketMergeWaves = QGA_BUCKET_MERGE_WAVES;
 
 template <int kW>
 void launch_bucket_merge(const MergeTable &tab, float *out, cudaStream_t stream)
 {
-    auto kernel = dequant_accumulate_2bit_bucket_kernel<kW>;
-    const int resident = resident_blocks(kernel, kThreads, occ_ab[kW]);
-    kernel<<<grid_for(tab.total_chunks, resident, kBucketMergeWaves), kThreads, 0, stream>>>(tab, out);
+    if constexpr (kW > 0) {
+        auto kernel = merge_2bit_table_bucket_kernel<kW>;
+        const int resident = resident_blocks(kernel, kThreads, occ_ab[kW]);
+        kernel<<<grid_for(tab.total_chunks, resident, kBucketMergeWaves), kThreads, 0, stream>>>(tab, out);
+    } else {
+        auto kernel = dequant_accumulate_2bit_bucket_kernel<0>;
+        const int resident = resident_blocks(kernel, kThreads, occ_ab[0]);
+        kernel<<<grid_for(tab.total_chunks, resident, kBucketMergeWaves), kThreads, 0, stream>>>(tab, out);
+    }
 }
 
 void launch_bucket_merge_any(const MergeTable &tab, float *out, cudaStream_t stream)

@@ -98,17 +98,94 @@ __global__ void __launch_bounds__(kThreads, QGA_LOCAL_REDUCE_MIN_BLOCKS)
     }
 }
 
+// W <= 8: the same step with the merge through the table of all 3^W sums
+// (build_sum_table, merge_2bit_table_*).  The received records' words of a
+// slice are loaded first, so they are in flight while the lane quantizes
+// its own words; the own word goes from the register straight into the
+// table index (it is stored too, and never read back).
+// Blocks per SM the table kernel's registers are fitted to: 3 spill (435 us
+// against 404 us at 2, n = 138M, W = 8).
+#ifndef QGA_LOCAL_REDUCE_TABLE_MIN_BLOCKS
+#define QGA_LOCAL_REDUCE_TABLE_MIN_BLOCKS 1
+#endif
+
+template <bool kVec, int kW>
+__global__ void __launch_bounds__(kThreads, QGA_LOCAL_REDUCE_TABLE_MIN_BLOCKS)
+    quantize_merge_2bit_table_kernel(const float *__restrict__ grad, float *__restrict__ residual,
+                                     int64_t n, float neg, float pos,
+                                     const __grid_constant__ RecordSet set, int own,
+                                     uint32_t *__restrict__ own_rec, float *__restrict__ out)
+{
+    __shared__ float s_neg[kW], s_pos[kW];
+    __shared__ float s_sum[Pow3<kW>::value];
+    __shared__ float4 s_stage[kWarpsPerBlock][kWarp * 4];
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        own_rec[0] = bits_from_f32(neg);
+        own_rec[1] = bits_from_f32(pos);
+        own_rec[2] = bits_from_f32(__ll2float_rn(n));
+    }
+    if (threadIdx.x < kW) {
+        const uint32_t *r = set.rec[threadIdx.x];
+        s_neg[threadIdx.x] = (int)threadIdx.x == own ? neg : f32_from_bits(r[0]);
+        s_pos[threadIdx.x] = (int)threadIdx.x == own ? pos : f32_from_bits(r[1]);
+    }
+    __syncthreads();
+    build_sum_table<kW>(s_sum, [&](int w) { return s_neg[w]; }, [&](int w) { return s_pos[w]; });
+    uint32_t *own_payload = own_rec + 3;
+    const int lane = threadIdx.x & (kWarp - 1);
+    const int64_t nwords = (n + 15) >> 4;
+    const int64_t slices = (n + kTableSliceElems - 1) / kTableSliceElems;
+    const int64_t stride = (int64_t)gridDim.x * kWarpsPerBlock;
+    for (int64_t sl = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5); sl < slices;
+         sl += stride) {
+        uint32_t wd[kTableSlots][kTableMaxWorkers];
+        merge_2bit_table_load<kW, kTableSlots>([&](int w) { return set.rec[w] + 3; }, nwords, sl, lane,
+                                               own, wd);
+#pragma unroll
+        for (int s = 0; s < kTableSlots; ++s) {
+            const int64_t k = (sl * kTableSlots + s) * kWarp + lane;
+            uint32_t word = 0u;
+            if (k < nwords) {
+                float g[16], r[16];
+                load_word<kVec>(grad, residual, n, k, g, r);
+                word = quantize_word<kVec>(residual, own_payload, n, k, neg, pos, g, r);
+            }
+            // the own worker's load was skipped (its slot holds 0); a register
+            // array is indexed by constants only, so the word is or-ed in by mask
+#pragma unroll
+            for (int w = 0; w < kW; ++w)
+                wd[s][w] |= word & (0u - (uint32_t)(w == own));
+        }
+        merge_2bit_table_store<kVec, kW, kTableSlots>(wd, s_sum, out, n, sl, lane,
+                                                      s_stage[threadIdx.x >> 5]);
+    }
+}
+
 std::atomic<int> occ_lr[2][9][64]; // [vec][kW][device]
+
+#ifndef QGA_LOCAL_REDUCE_WAVES
+#define QGA_LOCAL_REDUCE_WAVES 1
+#endif
 
 template <bool kVec, int kW>
 void launch_k(const float *grad, float *residual, int64_t n, float neg, float pos,
               const RecordSet &set, int W, int own, float *out, cudaStream_t stream)
 {
-    auto k = quantize_merge_2bit_kernel<kVec, kW>;
-    const int64_t slices = (n + kSliceElems - 1) / kSliceElems;
-    const unsigned grid = grid_for((slices + kWarpsPerBlock - 1) / kWarpsPerBlock,
-                                   resident_blocks(k, kThreads, occ_lr[kVec][kW]));
-    k<<<grid, kThreads, 0, stream>>>(grad, residual, n, neg, pos, set, W, own, out);
+    if constexpr (kW > 0) {
+        auto k = quantize_merge_2bit_table_kernel<kVec, kW>;
+        const int64_t slices = (n + kTableSliceElems - 1) / kTableSliceElems;
+        const unsigned grid = grid_for((slices + kWarpsPerBlock - 1) / kWarpsPerBlock,
+                                       resident_blocks(k, kThreads, occ_lr[kVec][kW]),
+                                       QGA_LOCAL_REDUCE_WAVES);
+        k<<<grid, kThreads, 0, stream>>>(grad, residual, n, neg, pos, set, own,
+                                         const_cast<uint32_t *>(set.rec[own]), out);
+    } else {
+        auto k = quantize_merge_2bit_kernel<kVec, 0>;
+        const int64_t slices = (n + kSliceElems - 1) / kSliceElems;
+        const unsigned grid = grid_for((slices + kWarpsPerBlock - 1) / kWarpsPerBlock,
+                                       resident_blocks(k, kThreads, occ_lr[kVec][0]));
+        k<<<grid, kThreads, 0, stream>>>(grad, residual, n, neg, pos, set, W, own, out);
+    }
 }
 
 template <bool kVec>

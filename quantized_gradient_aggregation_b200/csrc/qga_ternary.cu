@@ -280,12 +280,114 @@ __global__ void __launch_bounds__(kThreads)
     }
 }
 
+// ------------------------------------------------------ merge by sum table --
+// W <= 8: the merge through the table of all 3^W sums (build_sum_table in
+// qga_2bit_tiles.cuh: entry sum_k d_k 3^k holds the definition's sum of the
+// workers' code values, d_k the trit of worker k).  A lane owns one payload
+// word (20 elements) and turns every worker's 4 bytes into trits without
+// a lookup table: two bytes at a time in 16-bit lanes, floor(v / 3) =
+// (171 v) >> 9 (exact for v < 256), trit = v - 3 floor(v / 3), four times;
+// the leading trit is taken mod 3 like every other (a byte above 242 never
+// occurs in a record).  The trits of worker k, times 4 3^k, accumulate into
+// the byte offsets of the table entries (at most 4 * 6560 < 2^16).
+__device__ __forceinline__ uint32_t div3_16(uint32_t v) // two 16-bit lanes, each below 256
+{
+    return ((v * 171u) >> 9) & 0x007F007Fu;
+}
+
+// acc[i]: table offsets of trit i (0 = most significant) of the two bytes in
+// the lanes of v, plus 4 3^k times worker k's trits.
+__device__ __forceinline__ void add_trits(uint32_t v, uint32_t weight, uint32_t (&acc)[5])
+{
+    const uint32_t q1 = div3_16(v), q2 = div3_16(q1), q3 = div3_16(q2), q4 = div3_16(q3);
+    acc[4] += (v - 3u * q1) * weight;
+    acc[3] += (q1 - 3u * q2) * weight;
+    acc[2] += (q2 - 3u * q3) * weight;
+    acc[1] += (q3 - 3u * q4) * weight;
+    acc[0] += (q4 - 3u * ((q4 >> 1) & q4 & 0x00010001u)) * weight; // 3 -> 0
+}
+
+// Words per lane of a table-merge tile (build-time setting; the default is
+// the measured best): lane l owns words l, 32 + l, ... and loads all of them,
+// of every worker, before using any.
+#ifndef QGA_TERNARY_TABLE_SLOTS
+#define QGA_TERNARY_TABLE_SLOTS 2
+#endif
+constexpr int kTernarySlots = QGA_TERNARY_TABLE_SLOTS;
+
+template <bool kVec, int kW>
+__global__ void __launch_bounds__(kThreads)
+    merge_ternary_table_kernel(const __grid_constant__ RecordSet set, float *__restrict__ out, int64_t n)
+{
+    __shared__ float s_neg[kW], s_pos[kW];
+    __shared__ float s_sum[Pow3<kW>::value];
+    __shared__ float4 s_stage[kWarpsPerBlock][kWarp * 5];
+    if (threadIdx.x < kW) {
+        const uint32_t *r = set.rec[threadIdx.x];
+        s_neg[threadIdx.x] = f32_from_bits(r[0]);
+        s_pos[threadIdx.x] = f32_from_bits(r[1]);
+    }
+    __syncthreads();
+    build_sum_table<kW>(s_sum, [&](int w) { return s_neg[w]; }, [&](int w) { return s_pos[w]; });
+    const char *tb = reinterpret_cast<const char *>(s_sum);
+    float4 *stage = s_stage[threadIdx.x >> 5];
+    const int lane = threadIdx.x & (kWarp - 1);
+    const int64_t nwords = (n + 19) / 20;
+    const int64_t tiles = (nwords + kWarp * kTernarySlots - 1) / (kWarp * kTernarySlots);
+    for (int64_t t = warp_id(); t < tiles; t += warp_stride()) {
+        uint32_t words[kTernarySlots][kW];
+#pragma unroll
+        for (int sl = 0; sl < kTernarySlots; ++sl) {
+            const int64_t w = (t * kTernarySlots + sl) * kWarp + lane;
+#pragma unroll
+            for (int k = 0; k < kW; ++k)
+                words[sl][k] = w < nwords ? ld_stream_u32(set.rec[k] + 3 + w) : 0u;
+        }
+#pragma unroll
+        for (int sl = 0; sl < kTernarySlots; ++sl) {
+            // lanes: ev = bytes 0 and 2 of the word, od = bytes 1 and 3
+            uint32_t ev[5] = {}, od[5] = {};
+            uint32_t weight = 4u;
+#pragma unroll
+            for (int k = 0; k < kW; ++k) {
+                add_trits(words[sl][k] & 0x00FF00FFu, weight, ev);
+                add_trits((words[sl][k] >> 8) & 0x00FF00FFu, weight, od);
+                weight *= 3u;
+            }
+            // byte b of the word holds elements 5b .. 5b + 4 (trit i = element 5b + i)
+            float v[20];
+#pragma unroll
+            for (int i = 0; i < 5; ++i) {
+                v[i] = *reinterpret_cast<const float *>(tb + (ev[i] & 0xFFFFu));   // byte 0
+                v[10 + i] = *reinterpret_cast<const float *>(tb + (ev[i] >> 16)); // byte 2
+                v[5 + i] = *reinterpret_cast<const float *>(tb + (od[i] & 0xFFFFu)); // byte 1
+                v[15 + i] = *reinterpret_cast<const float *>(tb + (od[i] >> 16));   // byte 3
+            }
+#pragma unroll
+            for (int c = 0; c < 5; ++c)
+                stage[5 * lane + c] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+            __syncwarp();
+            const int64_t g0 = (t * kTernarySlots + sl) * (kWarp * 5); // first group of this word slot
+#pragma unroll
+            for (int j = 0; j < 5; ++j) {
+                const int q = j * kWarp + lane; // group of 4 within the slot's 32 words
+                store_group<kVec>(out, n, g0 + q, stage[q]);
+            }
+            __syncwarp();
+        }
+    }
+}
+
 std::atomic<int> occ_tq[2][64], occ_td[2][2][9][64]; // td: [vec][merge][kW]
 
 // Grid waves (see grid_for), measured at n = 138M: quantize 287 / 253 / 247 /
 // 243 / 240 us at 1 / 8 / 16 / 32 / 128 waves; merge (W = 8) 206 / 199 / 206
 // / 224 us at 1 / 8 / 16 / 32.
 constexpr int kTernaryQuantizeWaves = 32, kTernaryDecodeWaves = 8;
+#ifndef QGA_TERNARY_TABLE_WAVES
+#define QGA_TERNARY_TABLE_WAVES 1
+#endif
+constexpr int kTernaryTableWaves = QGA_TERNARY_TABLE_WAVES;
 
 unsigned warps_grid(int64_t warp_items, int resident, int waves)
 {
@@ -296,10 +398,17 @@ template <bool kVec, bool kMerge, int kW>
 void launch_decode_k(const RecordSet &set, int W, float *out, int64_t n, cudaStream_t stream)
 {
     const int64_t tiles = ((n + 19) / 20 + kWarp - 1) / kWarp;
-    auto k = decode_ternary_kernel<kVec, kMerge, kW>;
-    k<<<warps_grid(tiles, resident_blocks(k, kThreads, occ_td[kVec][kMerge][kW]), kTernaryDecodeWaves),
-        kThreads, 0,
-        stream>>>(set, W, out, n);
+    if constexpr (kMerge && kW > 0) {
+        auto k = merge_ternary_table_kernel<kVec, kW>;
+        const int64_t table_tiles = ((n + 19) / 20 + kWarp * kTernarySlots - 1) / (kWarp * kTernarySlots);
+        k<<<warps_grid(table_tiles, resident_blocks(k, kThreads, occ_td[kVec][kMerge][kW]),
+                       kTernaryTableWaves),
+            kThreads, 0, stream>>>(set, out, n);
+    } else {
+        auto k = decode_ternary_kernel<kVec, kMerge, kW>;
+        k<<<warps_grid(tiles, resident_blocks(k, kThreads, occ_td[kVec][kMerge][kW]), kTernaryDecodeWaves),
+            kThreads, 0, stream>>>(set, W, out, n);
+    }
 }
 
 template <bool kVec>

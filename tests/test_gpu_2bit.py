@@ -175,6 +175,33 @@ def test_dequant_accumulate(W, n):
     assert same_bits_f32(got, want), first_diff(got, want)
 
 
+@pytest.mark.parametrize("W", [1, 2, 5, 8, 9])
+def test_dequant_accumulate_code_11_reads_as_zero(W):
+    """Records holding the unused code 11 (never written by a quantize): it
+    reads as +0 in the merge, for every worker count (the table merge clears
+    it before forming an index, the per-worker merge decodes it as 0)."""
+    n = 4099
+    rng = np.random.default_rng(W)
+    recs = [_random_record(n, -float(a), float(b), 77 * w + W, with_code_11=True)
+            for w, (a, b) in enumerate(rng.uniform(0.01, 2.0, (W, 2)).astype(np.float32))]
+    out = torch.empty(n, device=DEV)
+    qga().qga_dequant_accumulate_2bit([_dev_words(r) for r in recs], out)
+    want = oracle.dequant_accumulate_2bit(recs, n)
+    assert same_bits_f32(f32(out), want), first_diff(f32(out), want)
+
+
+@pytest.mark.parametrize("W", [2, 8])
+def test_dequant_accumulate_shared_and_signed_zero_thresholds(W):
+    """Thresholds shared by all workers, and -0 as a negative threshold
+    (code 10 then adds -0, which leaves a +0 sum at +0)."""
+    n = 1000
+    recs = [_random_record(n, -0.0 if w % 2 else -0.5, 0.5, 5 * w) for w in range(W)]
+    out = torch.empty(n, device=DEV)
+    qga().qga_dequant_accumulate_2bit([_dev_words(r) for r in recs], out)
+    want = oracle.dequant_accumulate_2bit(recs, n)
+    assert same_bits_f32(f32(out), want), first_diff(f32(out), want)
+
+
 def test_resnet50_four_workers_full():
     """ResNet-50-sized gradient, 4 workers with their own seeds and
     residuals: every word, residual and merged value checked."""
