@@ -41,6 +41,7 @@ METRIC = "2-bit quantize+residual+pack Gelem/s and HBM GB/s (% of peak), n=138M 
 WORKLOAD = "vgg16-8w"
 QUANT_BYTES_PER_ELEM = 12.25        # read g 4 + read r 4 + write r 4 + write codes 0.25
 FALLBACK_HBM_GBS = 6650.0
+TS_PAIRS = ((4, 8), (2, 4))          # QSGD-MN-TS rows: (coarse bits, fine bits)
 
 # dram__bytes_read.sum + dram__bytes_write.sum per element of one full-size
 # launch of the quantize kernel (profiles/quantize_2bit_kernel_fp32_vgg16.md),
@@ -57,6 +58,8 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["qga", "reference"], default="qga")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--reduce-form", choices=["pair", "fused"], default="pair",
+                   help="the reducing worker's step: quantize + merge (pair) or one fused launch")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-rows", action="store_true",
                    help="skip the per-kernel timings of the other hot-path rows")
@@ -65,6 +68,10 @@ def parse_args():
     p.add_argument("--iterations", type=int, default=None, help="resident gradient sets")
     p.add_argument("--rows-scale", type=int, default=1,
                    help="divide the per-row workloads' sizes by this (profiler captures)")
+    p.add_argument("--rows-reps", type=int, default=20,
+                   help="timed launches per row (1 with --rows-warmup 0: each row kernel once, "
+                        "for profiler captures)")
+    p.add_argument("--rows-warmup", type=int, default=3)
     return p.parse_args()
 
 
@@ -115,14 +122,14 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def workload_config(w, n_gpus):
+def workload_config(w, n_gpus, reduce_form="pair"):
+    last = (f"then worker 0 (the reducing worker) quantizes its own gradient and all {w.workers} "
+            "records are merged" + (" in one launch" if reduce_form == "fused" else ""))
     return {
         "workload": (f"{w.name}: W={w.workers} simulated workers x n={w.n:,} fp32, "
                      f"g~Laplace(0,{w.scale:g}) (seeded synthetic, {w.iterations} iterations "
                      f"resident and cycled), residual carried, thresholds {w.neg_thr:g}/{w.pos_thr:g}; "
-                     f"step = quantize of workers 1..{w.workers - 1}, then worker 0 (the reducing "
-                     f"worker) quantizes its own gradient and merges all {w.workers} records in one "
-                     "launch"),
+                     f"step = quantize of workers 1..{w.workers - 1}, {last}"),
         "n": w.n,
         "workers": w.workers,
         "l2": "every buffer (553 MB per gradient) is larger than the 126 MB L2; no flush",
@@ -318,14 +325,28 @@ def run_qga(args, rank, world, local_rank):
         if st:
             raise q.QGAError(st, "qga_quantize_2bit")
 
-    def reduce(it):
+    def reduce_fused(it):
         # worker 0 is the reducing worker ([MX] Local kvstore): its own quantize
-        # and the merge of all W records are one launch
+        # and the merge of all W records in one launch
         st = L.qga_quantize_merge_2bit(ctypes.c_void_p(grads[it][0].data_ptr()),
                                        ctypes.c_void_p(res[0].data_ptr()), n, neg, pos, cpp, W, 0,
                                        ctypes.c_void_p(out.data_ptr()), sp)
         if st:
             raise q.QGAError(st, "qga_quantize_merge_2bit")
+
+    def reduce_pair(it):
+        # the same results from two launches: worker 0's quantize, then the merge
+        quant(it, 0)
+        st = L.qga_dequant_accumulate_2bit(cpp, W, ctypes.c_void_p(out.data_ptr()), n, sp)
+        if st:
+            raise q.QGAError(st, "qga_dequant_accumulate_2bit")
+
+    # The reducing worker's step (both forms give the same bits) is timed in
+    # the form given by --reduce-form: by default the pair, measured faster on
+    # B200 (391.6 against 404.4 us at n = 138M, W = 8).  Both forms are also
+    # timed alone after the timed region and reported.
+    reduce_form = args.reduce_form
+    reduce = reduce_fused if reduce_form == "fused" else reduce_pair
 
     def barrier():
         if world > 1:
@@ -369,12 +390,15 @@ def run_qga(args, rank, world, local_rank):
     merge_ms = statistics.fmean(a.elapsed_time(b) for a, b in m_ev)
     total_ms, quant_ms, merge_ms = max_over_ranks([total_ms, quant_ms, merge_ms], world, dev)
 
+    trial = {}
+    for name, fn in (("fused", reduce_fused), ("pair", reduce_pair)):
+        trial[name] = _time_launches(stream, lambda fn=fn: fn(0), 10, nvtx="reducing_worker_" + name) * 1e6
     e2e = None if args.no_e2e else run_e2e(args, w, grads[0], res, comprs, out, quant, reduce,
-                                           stream, world, dev)
+                                           stream, world, dev, reduce_form)
     del grads, res, comprs, out
     torch.cuda.empty_cache()
-    rows = None if args.no_rows else time_rows(dev, stream, measured_peaks()[0],
-                                               scale=max(1, args.rows_scale))
+    rows = None if args.no_rows else time_rows(dev, stream, measured_peaks()[0], reps=args.rows_reps,
+                                               scale=max(1, args.rows_scale), warmup=args.rows_warmup)
 
     if rank != 0:
         return
@@ -390,7 +414,7 @@ def run_qga(args, rank, world, local_rank):
         "ms_per_step": total_ms / K,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded Laplace(0,1e-3) gradients generated on the GPU)",
-        "config": workload_config(w, world),
+        "config": workload_config(w, world, reduce_form),
         "roofline": {"bound": "hbm", "kernel": "qga_quantize_2bit (quantize_2bit_words_kernel)",
                      "achieved": quant_gbs, "peak": peak, "unit": "GB/s", "frac": quant_gbs / peak,
                      "peak_source": f"{peak_kind} HBM copy rate",
@@ -401,13 +425,17 @@ def run_qga(args, rank, world, local_rank):
             "quantize_2bit": {"us": quant_ms * 1e3, "gelem_s": n / (quant_ms * 1e-3) / 1e9,
                               "gb_s": quant_gbs, "frac_of_peak": quant_gbs / peak,
                               "frac_of_8TBs": quant_gbs / 8000.0},
-            "quantize_merge_2bit_w8": {"us": merge_ms * 1e3,
+            "reducing_worker_step_w8": {"us": merge_ms * 1e3, "form": reduce_form,
                                        "gelem_s": n / (merge_ms * 1e-3) / 1e9,
                                        "gb_s": merge_gbs, "frac_of_peak": merge_gbs / peak,
                                        "frac_of_8TBs": merge_gbs / 8000.0,
                                        "bytes_per_elem": QUANT_BYTES_PER_ELEM + 0.25 * (W - 1) + 4},
         },
-        "gpu_launches": K * W,
+        "gpu_launches": K * (W + (reduce_form == "pair")),
+        "reducing_worker_step": {"timed_form": reduce_form,
+                                 "alone_us_after_timed_region": trial,
+                                 "forms": {"fused": "qga_quantize_merge_2bit (one launch)",
+                                           "pair": "qga_quantize_2bit + qga_dequant_accumulate_2bit"}},
         "clocks": clocks,
         "csrc": csrc_hash(),
         "quantize_sources": csrc_hash(QUANT_SOURCES),
@@ -422,18 +450,21 @@ def run_qga(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
-def _time_launches(stream, fn, reps, warmup=3):
+def _time_launches(stream, fn, reps, warmup=3, nvtx="row"):
     """Average device time of fn() (one or more kernel launches) over reps,
-    CUDA events on the launching stream."""
+    CUDA events on the launching stream.  The timed launches sit in an NVTX
+    range named ``nvtx`` (a profiler can select them by it)."""
     import torch
     for _ in range(warmup):
         fn()
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.nvtx.range_push(nvtx)
     a.record(stream)
     for _ in range(reps):
         fn()
     b.record(stream)
+    torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     return a.elapsed_time(b) / reps * 1e-3
 
@@ -447,7 +478,7 @@ def _row(seconds, elems, bytes_per_elem, peak, launches, **extra):
     return d
 
 
-def time_rows(dev, stream, peak, reps=20, scale=1):
+def time_rows(dev, stream, peak, reps=20, scale=1, warmup=3):
     """Device time of every other row of the hot path, each on its own
     workload at full size (inputs resident, larger than L2); ``scale`` > 1
     shrinks the flat workloads for profiler captures only."""
@@ -473,24 +504,32 @@ def time_rows(dev, stream, peak, reps=20, scale=1):
     q.qga_quantize_2bit(g, r, c, w.neg_thr, w.pos_thr)
     out = torch.empty(n, device=dev)
     t = _time_launches(stream, lambda: ok(L.qga_dequantize_2bit(vp(c.data_ptr()), vp(out.data_ptr()),
-                                                                n, sp), "dequantize"), reps)
-    rows["dequantize_2bit"] = _row(t, n, 4.25, peak, reps + 3, workload=f"vgg16 record, n={n:,}")
+                                                                n, sp), "dequantize"), reps, warmup)
+    rows["dequantize_2bit"] = _row(t, n, 4.25, peak, reps + warmup, workload=f"vgg16 record, n={n:,}")
 
     # the reducing worker's fused step: quantize worker 0, merge 8 records
-    others = [c.clone() for _ in range(w.workers - 1)]
+    # (the other workers' records from their own gradients)
+    others = []
+    for k in range(1, w.workers):
+        gk = workloads.gradient(w, k, 0, device=dev, n=n)
+        rk = torch.zeros(n, device=dev)
+        ck = torch.empty_like(c)
+        q.qga_quantize_2bit(gk, rk, ck, w.neg_thr, w.pos_thr)
+        others.append(ck)
+        del gk, rk
     c_own = torch.empty_like(c)
     rarr = (ctypes.c_void_p * w.workers)(*[x.data_ptr() for x in [c_own] + others])
     rp = ctypes.cast(rarr, ctypes.POINTER(ctypes.c_void_p))
     t = _time_launches(stream, lambda: ok(L.qga_quantize_merge_2bit(
         vp(g.data_ptr()), vp(r.data_ptr()), n, w.neg_thr, w.pos_thr, rp, w.workers, 0,
-        vp(out.data_ptr()), sp), "quantize_merge"), reps)
+        vp(out.data_ptr()), sp), "quantize_merge"), reps, warmup)
     rows["quantize_merge_2bit_w8_alone"] = _row(t, n, 12.25 + 0.25 * (w.workers - 1) + 4, peak,
-                                                reps + 3,
+                                                reps + warmup,
                                                 workload=f"vgg16 worker 0 + 7 received records, n={n:,}")
     # the merge alone (A8): 8 records
     t = _time_launches(stream, lambda: ok(L.qga_dequant_accumulate_2bit(
-        rp, w.workers, vp(out.data_ptr()), n, sp), "merge"), reps)
-    rows["dequant_accumulate_2bit_w8"] = _row(t, n, 0.25 * w.workers + 4, peak, reps + 3,
+        rp, w.workers, vp(out.data_ptr()), n, sp), "merge"), reps, warmup)
+    rows["dequant_accumulate_2bit_w8"] = _row(t, n, 0.25 * w.workers + 4, peak, reps + warmup,
                                               workload=f"8 records of n={n:,}")
     del c, others, c_own
 
@@ -498,15 +537,18 @@ def time_rows(dev, stream, peak, reps=20, scale=1):
     ct = [torch.empty(q.qga_ternary_words(n), dtype=torch.int32, device=dev) for _ in range(w.workers)]
     t = _time_launches(stream, lambda: ok(L.qga_quantize_ternary(
         vp(g.data_ptr()), vp(r.data_ptr()), vp(ct[0].data_ptr()), n, w.neg_thr, w.pos_thr, sp),
-        "quantize_ternary"), reps)
-    rows["quantize_ternary"] = _row(t, n, 12.2, peak, reps + 3, workload=f"vgg16 gradient, n={n:,}")
+        "quantize_ternary"), reps, warmup)
+    rows["quantize_ternary"] = _row(t, n, 12.2, peak, reps + warmup, workload=f"vgg16 gradient, n={n:,}")
     for k in range(1, w.workers):
-        ct[k].copy_(ct[0])
+        gk = workloads.gradient(w, k, 0, device=dev, n=n)
+        rk = torch.zeros(n, device=dev)
+        q.qga_quantize_ternary(gk, rk, ct[k], w.neg_thr, w.pos_thr)
+        del gk, rk
     tarr = (ctypes.c_void_p * w.workers)(*[cc.data_ptr() for cc in ct])
     tp = ctypes.cast(tarr, ctypes.POINTER(ctypes.c_void_p))
     t = _time_launches(stream, lambda: ok(L.qga_dequant_accumulate_ternary(
-        tp, w.workers, vp(out.data_ptr()), n, sp), "merge_ternary"), reps)
-    rows["dequant_accumulate_ternary_w8"] = _row(t, n, 0.2 * w.workers + 4, peak, reps + 3,
+        tp, w.workers, vp(out.data_ptr()), n, sp), "merge_ternary"), reps, warmup)
+    rows["dequant_accumulate_ternary_w8"] = _row(t, n, 0.2 * w.workers + 4, peak, reps + warmup,
                                                  workload=f"8 dense records of n={n:,}")
     del g, r, out, ct
 
@@ -532,8 +574,8 @@ def time_rows(dev, stream, peak, reps=20, scale=1):
            "quantize_bucket")
     for k in range(wb.workers):
         quant_bucket(k)
-    t = _time_launches(stream, quant_bucket, reps)
-    rows["quantize_2bit_bucket_bf16"] = _row(t, total, 10.25, peak, reps + 3 + wb.workers,
+    t = _time_launches(stream, quant_bucket, reps, warmup)
+    rows["quantize_2bit_bucket_bf16"] = _row(t, total, 10.25, peak, reps + warmup + wb.workers,
                                              workload="BERT-Base bucket, 197 bf16 tensors, "
                                                       "109,480,704 elements")
     out = torch.empty(total, device=dev)
@@ -541,8 +583,8 @@ def time_rows(dev, stream, peak, reps=20, scale=1):
     pp = ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p))
     nn = (ctypes.c_int64 * T)(*sizes)
     t = _time_launches(stream, lambda: ok(L.qga_dequant_accumulate_2bit_bucket(
-        pp, wb.workers, nn, T, vp(out.data_ptr()), sp), "merge_bucket"), reps)
-    rows["dequant_accumulate_2bit_bucket_w4"] = _row(t, total, 0.25 * wb.workers + 4, peak, reps + 3,
+        pp, wb.workers, nn, T, vp(out.data_ptr()), sp), "merge_bucket"), reps, warmup)
+    rows["dequant_accumulate_2bit_bucket_w4"] = _row(t, total, 0.25 * wb.workers + 4, peak, reps + warmup,
                                                      workload="BERT-Base bucket, 4 workers")
     del keep, comprs, out, tables
 
@@ -553,8 +595,8 @@ def time_rows(dev, stream, peak, reps=20, scale=1):
     cb = torch.empty(q.qga_2bit_words(total), dtype=torch.int32, device=dev)
     t = _time_launches(stream, lambda: ok(L.qga_quantize_2bit_bf16(
         vp(gb.data_ptr()), vp(rb.data_ptr()), vp(cb.data_ptr()), total, neg[0], pos[0], sp),
-        "quantize_bf16"), reps)
-    rows["quantize_2bit_bf16"] = _row(t, total, 10.25, peak, reps + 3,
+        "quantize_bf16"), reps, warmup)
+    rows["quantize_2bit_bf16"] = _row(t, total, 10.25, peak, reps + warmup,
                                       workload=f"one flat bf16 gradient, n={total:,}")
     del gb, rb, cb
 
@@ -566,8 +608,8 @@ def time_rows(dev, stream, peak, reps=20, scale=1):
     garr = (ctypes.c_void_p * Wq)(*[gg.data_ptr() for gg in grads])
     gp = ctypes.cast(garr, ctypes.POINTER(ctypes.c_void_p))
     t = _time_launches(stream, lambda: ok(L.qga_qsgd_mn_max(gp, Wq, nq, vp(M.data_ptr()), sp),
-                                          "qsgd_max"), reps)
-    rows["qsgd_mn_max_w8"] = _row(t, nq * Wq, 4.0, peak, reps + 3,
+                                          "qsgd_max"), reps, warmup)
+    rows["qsgd_mn_max_w8"] = _row(t, nq * Wq, 4.0, peak, reps + warmup,
                                   workload=f"8 x {nq:,} fp32 (0.1% outliers of 50)")
     out = torch.empty(nq, device=dev)
     for b in wq.bits:
@@ -579,24 +621,46 @@ def time_rows(dev, stream, peak, reps=20, scale=1):
                "qsgd_quantize")
         for k in range(Wq):
             quant_q(k)
-        t = _time_launches(stream, quant_q, reps)
-        rows[f"qsgd_mn_quantize_b{b}"] = _row(t, nq, 4 + b / 8, peak, reps + 3 + Wq,
+        t = _time_launches(stream, quant_q, reps, warmup)
+        rows[f"qsgd_mn_quantize_b{b}"] = _row(t, nq, 4 + b / 8, peak, reps + warmup + Wq,
                                               workload=f"{nq:,} fp32, b={b}")
         carr = (ctypes.c_void_p * Wq)(*[cc.data_ptr() for cc in cq])
         cp = ctypes.cast(carr, ctypes.POINTER(ctypes.c_void_p))
         t = _time_launches(stream, lambda: ok(L.qga_qsgd_mn_dequant_accumulate(
-            cp, Wq, vp(out.data_ptr()), nq, b, sp), "qsgd_merge"), reps)
-        rows[f"qsgd_mn_dequant_accumulate_b{b}_w8"] = _row(t, nq, Wq * b / 8 + 4, peak, reps + 3,
+            cp, Wq, vp(out.data_ptr()), nq, b, sp), "qsgd_merge"), reps, warmup)
+        rows[f"qsgd_mn_dequant_accumulate_b{b}_w8"] = _row(t, nq, Wq * b / 8 + 4, peak, reps + warmup,
                                                           workload=f"8 records of {nq:,}, b={b}")
         del cq
+
+    # QSGD-MN-TS: coarse scale M with b1 bits, fine scale M / s1 with b2 bits
+    for b1, b2 in TS_PAIRS:
+        words = q.qga_qsgd_mnts_words(nq, b1, b2)
+        ct = [torch.empty(words, dtype=torch.int32, device=dev) for _ in range(Wq)]
+
+        def quant_ts(k=0, b1=b1, b2=b2, ct=ct):
+            ok(L.qga_qsgd_mnts_quantize(vp(grads[k].data_ptr()), vp(ct[k].data_ptr()), nq, b1, b2,
+                                        workloads.QSGD_SEED_BASE + k, vp(M.data_ptr()), sp),
+               "qsgd_mnts_quantize")
+        for k in range(Wq):
+            quant_ts(k)
+        t = _time_launches(stream, quant_ts, reps, warmup)
+        rows[f"qsgd_mnts_quantize_b{b1}_{b2}"] = _row(t, nq, 4 + (b1 + b2) / 8, peak, reps + warmup + Wq,
+                                                      workload=f"{nq:,} fp32, b1={b1}, b2={b2}")
+        carr = (ctypes.c_void_p * Wq)(*[cc.data_ptr() for cc in ct])
+        cp = ctypes.cast(carr, ctypes.POINTER(ctypes.c_void_p))
+        t = _time_launches(stream, lambda: ok(L.qga_qsgd_mnts_dequant_accumulate(
+            cp, Wq, vp(out.data_ptr()), nq, b1, b2, sp), "qsgd_mnts_merge"), reps, warmup)
+        rows[f"qsgd_mnts_dequant_accumulate_b{b1}_{b2}_w8"] = _row(
+            t, nq, Wq * (b1 + b2) / 8 + 4, peak, reps + warmup, workload=f"8 records of {nq:,}, b1={b1}, b2={b2}")
+        del ct
 
     # GRandK-MaxNorm: the same gradients, K = 10000 shared coordinates
     K = workloads.GRANDK_K
     index = torch.from_numpy(workloads.grandk_index(nq, K)).to(dev)
     ip = vp(index.data_ptr())
     t = _time_launches(stream, lambda: ok(L.qga_grandk_mn_max(gp, Wq, nq, ip, K, vp(M.data_ptr()), sp),
-                                          "grandk_max"), reps)
-    rows["grandk_mn_max_w8"] = _row(t, K * Wq, 4.0, peak, reps + 3, bound="latency",
+                                          "grandk_max"), reps, warmup)
+    rows["grandk_mn_max_w8"] = _row(t, K * Wq, 4.0, peak, reps + warmup, bound="latency",
                                     workload=f"8 x {nq:,} fp32, K = {K:,} kept coordinates")
     for b in wq.bits:
         ck = [torch.empty(q.qga_qsgd_words(K, b), dtype=torch.int32, device=dev) for _ in range(Wq)]
@@ -607,16 +671,16 @@ def time_rows(dev, stream, peak, reps=20, scale=1):
                "grandk_quantize")
         for k in range(Wq):
             quant_k(k)
-        t = _time_launches(stream, quant_k, reps)
-        rows[f"grandk_mn_quantize_b{b}"] = _row(t, K, 4 + 8 + b / 8, peak, reps + 3 + Wq,
+        t = _time_launches(stream, quant_k, reps, warmup)
+        rows[f"grandk_mn_quantize_b{b}"] = _row(t, K, 4 + 8 + b / 8, peak, reps + warmup + Wq,
                                                 bound="latency", workload=f"K = {K:,} of {nq:,}, b={b}")
         carr = (ctypes.c_void_p * Wq)(*[cc.data_ptr() for cc in ck])
         cp = ctypes.cast(carr, ctypes.POINTER(ctypes.c_void_p))
         # the merge clears the n-element result (cudaMemsetAsync), then scatters K values
         t = _time_launches(stream, lambda: ok(L.qga_grandk_mn_dequant_accumulate(
-            cp, Wq, ip, K, vp(out.data_ptr()), nq, b, sp), "grandk_merge"), reps)
+            cp, Wq, ip, K, vp(out.data_ptr()), nq, b, sp), "grandk_merge"), reps, warmup)
         rows[f"grandk_mn_dequant_accumulate_b{b}_w8"] = _row(
-            t, nq, 4 + (K * (8 + 4 + Wq * b / 8)) / nq, peak, reps + 3, bound="hbm (clear of out)",
+            t, nq, 4 + (K * (8 + 4 + Wq * b / 8)) / nq, peak, reps + warmup, bound="hbm (clear of out)",
             workload=f"8 records of K = {K:,}, out of {nq:,}")
         del ck
     del grads, out, index
@@ -624,7 +688,7 @@ def time_rows(dev, stream, peak, reps=20, scale=1):
     return rows
 
 
-def run_e2e(args, w, dev_grads, res, comprs, out, quant, reduce, stream, world, dev):
+def run_e2e(args, w, dev_grads, res, comprs, out, quant, reduce, stream, world, dev, reduce_form):
     """Same step with the gradients arriving from pinned host memory and the
     aggregate read back, copies inside the timed region.  Uploads run on one
     copy stream, so worker k's upload overlaps the quantize of the worker
@@ -685,8 +749,9 @@ def run_e2e(args, w, dev_grads, res, comprs, out, quant, reduce, stream, world, 
     (ms,) = max_over_ranks([a.elapsed_time(b)], world, dev)
     return {"value": job_gelem_per_s(world, W, n, K, ms), "unit": "Gelem/s",
             "h2d_bytes_per_step": W * n * 4, "d2h_bytes_per_step": n * 4, "steps": K,
-            "path": "pinned host gradients -> cudaMemcpyAsync (copy stream) -> qga_quantize_2bit x7 "
-                    "-> qga_quantize_merge_2bit (worker 0) -> pinned host aggregate (download stream)"}
+            "path": ("pinned host gradients -> cudaMemcpyAsync (copy stream) -> qga_quantize_2bit x7 -> "
+                     + ("qga_quantize_2bit + qga_dequant_accumulate_2bit" if reduce_form == "pair"
+                        else "qga_quantize_merge_2bit") + " (worker 0) -> pinned host aggregate (download stream)")}
 
 
 def main():

@@ -173,6 +173,79 @@ __global__ void __launch_bounds__(kThreads)
     }
 }
 
+// The quantize in lane-owned words, for a 32-byte-aligned gradient: lane l
+// of warp t owns the 16 consecutive elements 16 (32 t + l) .. + 15 (two
+// 256-bit loads, the 4 Philox blocks of its 4 groups), forms their levels
+// with the fixed-point level (qsgd_level_lean) and packs its b / 2 record
+// words in registers: no shuffles and one check per lane.  A lane whose
+// check flags any element recomputes all 16 by the definition's operations.
+template <int B>
+__global__ void __launch_bounds__(kThreads)
+    qsgd_quantize_words_kernel(const float *__restrict__ grad, uint32_t *__restrict__ compr, int64_t n,
+                               uint32_t key0, uint32_t key1, const float *__restrict__ max_in)
+{
+    using L = Levels<B>;
+    constexpr int E = B - 1;
+    constexpr int kWords = B / 2; // record words per 16 elements
+    constexpr int kPer = 32 / B;  // elements per word
+    const float M = *max_in;
+    const bool fast = M > 0.0f && M <= FLT_MAX; // uniform over the grid
+    const float k = __fdiv_rn((float)L::s, M);
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        compr[0] = bits_from_f32(M);
+        compr[1] = bits_from_f32((float)B);
+        compr[2] = bits_from_f32(__ll2float_rn(n));
+    }
+    uint32_t *payload = compr + 3;
+    const int lane = threadIdx.x & (kWarp - 1);
+    const int64_t nwords = (n * B + 31) >> 5;
+    const int64_t runs = (n + 16 * kWarp - 1) / (16 * kWarp);
+    for (int64_t t = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5); t < runs;
+         t += (int64_t)gridDim.x * kWarpsPerBlock) {
+        const int64_t r = t * kWarp + lane; // this lane's run of 16 elements
+        const int64_t e0 = 16 * r;
+        float g[16];
+        if (e0 + 16 <= n) {
+            ld_stream_f8(grad + e0, g);
+            ld_stream_f8(grad + e0 + 8, g + 8);
+        } else {
+#pragma unroll
+            for (int p = 0; p < 16; ++p)
+                g[p] = e0 + p < n ? ld_stream_f1(grad + e0 + p) : 0.0f;
+        }
+        uint4 d[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int64_t gi = 4 * r + j;
+            d[j] = philox4x32_10(make_uint4((uint32_t)gi, (uint32_t)((uint64_t)gi >> 32), 0u, 0u), key0, key1);
+        }
+        const uint32_t x[16] = {d[0].x, d[0].y, d[0].z, d[0].w, d[1].x, d[1].y, d[1].z, d[1].w,
+                                d[2].x, d[2].y, d[2].z, d[2].w, d[3].x, d[3].y, d[3].z, d[3].w};
+        uint32_t w[kWords] = {};
+        uint32_t fmin = 0xFFFFFFFFu, tmax = 0u;
+#pragma unroll
+        for (int p = 0; p < 16; ++p) {
+            const uint32_t c = signed_code<B>(qsgd_level_lean<E>(g[p], k, x[p], fmin, tmax), g[p]);
+            w[p / kPer] |= c << (32 - B * (p % kPer + 1));
+        }
+        if (!fast || LeanLevel<E>::needs_exact(fmin, tmax, (uint32_t)L::s)) {
+#pragma unroll
+            for (int i = 0; i < kWords; ++i)
+                w[i] = 0u;
+#pragma unroll
+            for (int p = 0; p < 16; ++p) {
+                const uint32_t c = (uint32_t)qsgd_level_exact<B>(g[p], M, unit_draw(x[p])) & L::mask;
+                w[p / kPer] |= c << (32 - B * (p % kPer + 1));
+            }
+        }
+        // elements past n loaded as 0 have level 0, so their codes are 0
+#pragma unroll
+        for (int i = 0; i < kWords; ++i)
+            if (r * kWords + i < nwords)
+                st_stream_u32(payload + r * kWords + i, w[i]);
+    }
+}
+
 // ----------------------------------------------------------------- merge ----
 // Integer sum of the W workers' levels a whole record word at a time (Swar,
 // swar_add_word in qga_qsgd_level.cuh).  A thread owns whole words: word l of
@@ -276,6 +349,10 @@ __global__ void __launch_bounds__(kThreads)
 
 std::atomic<int> occ_max[64];
 std::atomic<int> occ_q[3][2][64];
+std::atomic<int> occ_qw[3][64];
+#ifndef QGA_QSGD_LANE_WORDS
+#define QGA_QSGD_LANE_WORDS 1
+#endif
 std::atomic<int> occ_m[3][2][64];
 
 int bits_slot(int bits) { return bits == 2 ? 0 : (bits == 4 ? 1 : (bits == 8 ? 2 : -1)); }
@@ -285,7 +362,10 @@ int bits_slot(int bits) { return bits == 2 ? 0 : (bits == 4 ? 1 : (bits == 8 ? 2
 // merge (W = 8) b = 2 150 / 148 / 148, b = 4 231 / 206 / 201, b = 8 263 / 268 /
 // 266 us at 1 / 8 / 16 waves.  The max stays persistent (one atomic per block;
 // 606 / 602 / 606 / 696 us at 1 / 8 / 16 / 32).
-constexpr int kQsgdQuantizeWaves = 8;
+#ifndef QGA_QSGD_QUANTIZE_WAVES
+#define QGA_QSGD_QUANTIZE_WAVES 8
+#endif
+constexpr int kQsgdQuantizeWaves = QGA_QSGD_QUANTIZE_WAVES;
 template <int B> constexpr int kQsgdMergeWaves = B == 8 ? 1 : 16;
 
 template <int B>
@@ -309,7 +389,13 @@ void launch_quantize(const float *grad, uint32_t *compr, int64_t n, uint64_t see
 {
     const uint32_t k0 = (uint32_t)seed, k1 = (uint32_t)(seed >> 32);
     const int s = bits_slot(B);
-    if (aligned(grad, 16)) {
+    if (QGA_QSGD_LANE_WORDS && aligned(grad, 32)) {
+        auto k = qsgd_quantize_words_kernel<B>;
+        const int64_t runs = (n + 16 * kWarp - 1) / (16 * kWarp);
+        k<<<grid_for((runs + kWarpsPerBlock - 1) / kWarpsPerBlock, resident_blocks(k, kThreads, occ_qw[s]),
+                     kQsgdQuantizeWaves),
+            kThreads, 0, stream>>>(grad, compr, n, k0, k1, M);
+    } else if (aligned(grad, 16)) {
         auto k = qsgd_quantize_kernel<B, true>;
         k<<<group_grid(n, resident_blocks(k, kThreads, occ_q[s][0])), kThreads, 0, stream>>>(
             grad, compr, n, k0, k1, M);

@@ -145,6 +145,45 @@ __device__ __forceinline__ int32_t qsgd_level_fixed(float g, float k, uint32_t s
     return (int32_t)((level ^ sg) - sg);
 }
 
+// The same fixed-point level with one fused multiply-add and checks that
+// cost two integer min/max per element: X = fl(|g| k + 2^E) (a single
+// rounding, within half an ulp of the exact sum), T + 8 as above, and the
+// level floor(T / 2^F) with no cap.  A lane falls back to
+// qsgd_level_exact when, over its elements, the smallest fraction of T + 8
+// (shifted to the top bits) is below 16 units, or the largest T + 8 reaches
+// (s + 1) 2^F: a level above s (the cap case near |g| = M, or |g| > M),
+// and an infinite or NaN X all land there.  The error bound is that of
+// qsgd_level_fixed (the fused add only removes one rounding), so with the
+// same margin the two floors agree everywhere else.  2^E must exceed s.
+template <int E> struct LeanLevel {
+    static constexpr int F = 23 - E;
+    static constexpr uint32_t kOne = (127u + E) << 23;  // binary32 bits of 2^E
+    static __device__ __forceinline__ bool needs_exact(uint32_t fmin, uint32_t tmax, uint32_t s)
+    {
+        return fmin < (16u << (32 - F)) || tmax >= ((s + 1u) << F);
+    }
+};
+
+template <int E>
+__device__ __forceinline__ uint32_t qsgd_level_lean(float g, float k, uint32_t x, uint32_t &fmin,
+                                                    uint32_t &tmax)
+{
+    using Lx = LeanLevel<E>;
+    const float X = __fmaf_rn(fabsf(g), k, (float)(1 << E));
+    const uint32_t t8 = __float_as_uint(X) + (x >> (32 - Lx::F)) + (8u - Lx::kOne);
+    fmin = min(fmin, t8 << (32 - Lx::F));
+    tmax = max(tmax, t8);
+    return t8 >> Lx::F;
+}
+
+// The b-bit two's-complement code of a level of magnitude L with g's sign.
+template <int B>
+__device__ __forceinline__ uint32_t signed_code(uint32_t L, float g)
+{
+    const int32_t sgn = ((int32_t)__float_as_uint(g) >> 31) * 2 + 1; // -1 or +1
+    return (uint32_t)((int32_t)L * sgn) & ((1u << B) - 1u);
+}
+
 // ------------------------------------------------- integer sum of levels --
 // The merges add the W workers' levels a whole record word at a time.  XOR
 // with the sign bit of every b-bit field turns a two's-complement level q

@@ -22,10 +22,10 @@
 // Quantize: the one-scale kernel's tile geometry (a warp owns 128 groups of
 // 4 elements, lane l groups l, l+32, l+64, l+96; one Philox block per group),
 // the fixed-point level of qga_qsgd_level.cuh with E = max(b1, b2) - 1 and
-// the scale picked per element, and two packed outputs.  Merge: a lane owns
-// 16 consecutive elements, sums each scale's levels over the workers in SIMD
-// lanes of registers (swar_add_word), converts and scales them once and
-// stores its 16 results as two 256-bit rows.
+// the scale picked per element, and two packed outputs.  Merge: each scale's
+// levels summed over the workers in SIMD lanes of registers (swar_add_word)
+// in that sub-record's own coalesced layout, converted and scaled once, and
+// the two parts added in shared memory (see qsgd_ts_merge_kernel).
 
 #include <float.h>
 
@@ -163,49 +163,178 @@ __global__ void __launch_bounds__(kThreads)
     }
 }
 
-// ----------------------------------------------------------------- merge ----
-constexpr int kSpan = 16; // elements per lane
+// The quantize in lane-owned words, for a 32-byte-aligned gradient: lane l
+// of warp t owns the 16 consecutive elements 16 (32 t + l) .. + 15 (two
+// 256-bit loads, the 4 Philox blocks of its 4 groups) and packs their codes
+// into its b1 / 2 coarse and b2 / 2 fine record words in registers (no
+// shuffles, one check per lane).  The level: X = fl(|g| k + 2^E) in one
+// fused multiply-add with the element's scale, then as in
+// qsgd_level_fixed (cap at the scale's s; fall back when any fraction of
+// T + 8 is below 16 units or X >= 2^(E+1)).
+template <int B1, int B2>
+__global__ void __launch_bounds__(kThreads)
+    qsgd_ts_quantize_words_kernel(const float *__restrict__ grad, uint32_t *__restrict__ compr, int64_t n,
+                                  uint32_t key0, uint32_t key1, const float *__restrict__ max_in)
+{
+    using L1 = Levels<B1>;
+    using L2 = Levels<B2>;
+    constexpr int E = (B1 > B2 ? B1 : B2) - 1;
+    constexpr int F = 23 - E;
+    constexpr uint32_t kOne = (127u + E) << 23, kTwo = (128u + E) << 23;
+    constexpr int kWords1 = B1 / 2, kWords2 = B2 / 2, kPer1 = 32 / B1, kPer2 = 32 / B2;
+    const float M1 = *max_in;
+    const float M2 = __fdiv_rn(M1, (float)L1::s);
+    const bool fast = M2 > 0.0f && M1 <= FLT_MAX; // uniform over the grid
+    const float k1 = __fdiv_rn((float)L1::s, M1);
+    const float k2 = __fdiv_rn((float)L2::s, M2);
+    uint32_t *coarse = compr;
+    uint32_t *fine = compr + sub_words(n, B1);
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        coarse[0] = bits_from_f32(M1);
+        coarse[1] = bits_from_f32((float)B1);
+        coarse[2] = bits_from_f32(__ll2float_rn(n));
+        fine[0] = bits_from_f32(M2);
+        fine[1] = bits_from_f32((float)B2);
+        fine[2] = bits_from_f32(__ll2float_rn(n));
+    }
+    const int lane = threadIdx.x & (kWarp - 1);
+    const int64_t nwords1 = (n * B1 + 31) >> 5, nwords2 = (n * B2 + 31) >> 5;
+    const int64_t runs = (n + 16 * kWarp - 1) / (16 * kWarp);
+    for (int64_t t = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5); t < runs;
+         t += (int64_t)gridDim.x * kWarpsPerBlock) {
+        const int64_t r = t * kWarp + lane; // this lane's run of 16 elements
+        const int64_t e0 = 16 * r;
+        float g[16];
+        if (e0 + 16 <= n) {
+            ld_stream_f8(grad + e0, g);
+            ld_stream_f8(grad + e0 + 8, g + 8);
+        } else {
+#pragma unroll
+            for (int p = 0; p < 16; ++p)
+                g[p] = e0 + p < n ? ld_stream_f1(grad + e0 + p) : 0.0f;
+        }
+        uint4 d[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int64_t gi = 4 * r + j;
+            d[j] = philox4x32_10(make_uint4((uint32_t)gi, (uint32_t)((uint64_t)gi >> 32), 0u, 0u), key0, key1);
+        }
+        const uint32_t x[16] = {d[0].x, d[0].y, d[0].z, d[0].w, d[1].x, d[1].y, d[1].z, d[1].w,
+                                d[2].x, d[2].y, d[2].z, d[2].w, d[3].x, d[3].y, d[3].z, d[3].w};
+        uint32_t w1[kWords1] = {}, w2[kWords2] = {};
+        uint32_t fmin = 0xFFFFFFFFu, xmax = 0u;
+#pragma unroll
+        for (int p = 0; p < 16; ++p) {
+            const bool is_fine = fabsf(g[p]) <= M2;
+            const uint32_t xb = __float_as_uint(__fmaf_rn(fabsf(g[p]), is_fine ? k2 : k1, (float)(1 << E)));
+            const uint32_t t8 = xb + (x[p] >> (32 - F)) + (8u - kOne);
+            fmin = min(fmin, t8 << (32 - F));
+            xmax = max(xmax, xb);
+            const uint32_t lv = min(t8 >> F, is_fine ? (uint32_t)L2::s : (uint32_t)L1::s);
+            const int32_t q = (int32_t)lv * (((int32_t)__float_as_uint(g[p]) >> 31) * 2 + 1);
+            w1[p / kPer1] |= (is_fine ? 0u : ((uint32_t)q & L1::mask)) << (32 - B1 * (p % kPer1 + 1));
+            w2[p / kPer2] |= (is_fine ? ((uint32_t)q & L2::mask) : 0u) << (32 - B2 * (p % kPer2 + 1));
+        }
+        if (!fast || fmin < (16u << (32 - F)) || xmax >= kTwo) {
+#pragma unroll
+            for (int i = 0; i < kWords1; ++i)
+                w1[i] = 0u;
+#pragma unroll
+            for (int i = 0; i < kWords2; ++i)
+                w2[i] = 0u;
+#pragma unroll
+            for (int p = 0; p < 16; ++p) {
+                const float u = unit_draw(x[p]);
+                if (fabsf(g[p]) <= M2)
+                    w2[p / kPer2] |= ((uint32_t)qsgd_level_exact<B2>(g[p], M2, u) & L2::mask)
+                                     << (32 - B2 * (p % kPer2 + 1));
+                else
+                    w1[p / kPer1] |= ((uint32_t)qsgd_level_exact<B1>(g[p], M1, u) & L1::mask)
+                                     << (32 - B1 * (p % kPer1 + 1));
+            }
+        }
+        // elements past n loaded as 0 have level 0 on the fine scale and code 0
+#pragma unroll
+        for (int i = 0; i < kWords1; ++i)
+            if (r * kWords1 + i < nwords1)
+                st_stream_u32(coarse + 3 + r * kWords1 + i, w1[i]);
+#pragma unroll
+        for (int i = 0; i < kWords2; ++i)
+            if (r * kWords2 + i < nwords2)
+                st_stream_u32(fine + 3 + r * kWords2 + i, w2[i]);
+    }
+}
 
-// The biased level sums of a lane's 16 elements on one scale of b bits:
-// the span's b/2 words of every worker (payload word span * b/2 + i).
-template <int B>
-__device__ __forceinline__ void span_sums(const RecordSet &set, int W, int64_t payload_off, int64_t span,
-                                          int64_t nwords, uint32_t (&sum)[kSpan])
+// ----------------------------------------------------------------- merge ----
+// A warp owns chunks of 512 elements.  Each sub-record is summed in its own
+// coalesced layout: the chunk's 16 b words, lane l owning words l, 32 + l,
+// ... (b / 2 of them), the levels of all workers added in SIMD lanes of
+// registers (swar_add_word); each element's sum is converted exactly,
+// scaled once by that scale's step and written to the warp's 2 KB of shared
+// memory (the coarse part), or added there to the coarse part (the fine
+// part).  The 512 results then leave as coalesced 128-bit rows.
+constexpr int kChunk = 512;
+
+// One scale's part of a chunk: this lane's words c * 32 + lane (c < b / 2)
+// of the chunk's 16 b words, summed over the workers in SIMD lanes of
+// registers, converted exactly, scaled once by the scale's step and stored
+// to sv (the coarse part) or added to the value there (kAdd, the fine part).
+// Word c * 32 + lane holds the elements (c * 32 + lane) * 32 / b ...
+#ifndef QGA_TS_MERGE_BATCH
+#define QGA_TS_MERGE_BATCH 4
+#endif
+template <int B, bool kAdd>
+__device__ __forceinline__ void chunk_part(const RecordSet &set, int W, int64_t payload_off, int64_t chunk,
+                                           int64_t nwords, int lane, float step, float bias,
+                                           float *__restrict__ sv)
 {
     using S = Swar<B>;
-    constexpr int kWordsPerSpan = kSpan * B / 32;
-    uint32_t acc[kWordsPerSpan][S::kRegs] = {};
-    constexpr int kBatch = 4;
+    constexpr int kWords = B / 2;
+    constexpr int kBatch = QGA_TS_MERGE_BATCH;
+    uint32_t acc[kWords][S::kRegs] = {};
     for (int wb = 0; wb < W; wb += kBatch) {
-        uint32_t words[kBatch][kWordsPerSpan];
+        uint32_t words[kBatch][kWords];
 #pragma unroll
         for (int i = 0; i < kBatch; ++i)
 #pragma unroll
-            for (int c = 0; c < kWordsPerSpan; ++c) {
-                const int64_t k = span * kWordsPerSpan + c;
+            for (int c = 0; c < kWords; ++c) {
+                const int64_t k = chunk * (16 * B) + c * kWarp + lane;
                 words[i][c] = (wb + i < W && k < nwords) ? ld_stream_u32(set.rec[wb + i] + payload_off + k)
-                                                         : Swar<B>::kSign; // biased 0 of an absent worker
+                                                         : S::kSign; // the biased 0 of an absent level
             }
 #pragma unroll
         for (int i = 0; i < kBatch; ++i) {
             if (wb + i >= W) // warp-uniform
                 break;
 #pragma unroll
-            for (int c = 0; c < kWordsPerSpan; ++c)
+            for (int c = 0; c < kWords; ++c)
                 swar_add_word<B>(acc[c], words[i][c]);
         }
     }
 #pragma unroll
-    for (int c = 0; c < kWordsPerSpan; ++c)
+    for (int c = 0; c < kWords; ++c) {
+        float v[S::kFields];
 #pragma unroll
         for (int e = 0; e < S::kFields; ++e)
-            sum[c * S::kFields + e] = swar_field_sum<B>(acc[c], e);
+            v[e] = __fmul_rn(__fsub_rn(__uint_as_float(0x4B000000u | swar_field_sum<B>(acc[c], e)), bias), step);
+        float4 *dst = reinterpret_cast<float4 *>(sv + (c * kWarp + lane) * S::kFields);
+#pragma unroll
+        for (int q = 0; q < S::kFields / 4; ++q) {
+            float4 x = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+            if (kAdd) {
+                const float4 a = dst[q];
+                x = make_float4(__fadd_rn(a.x, x.x), __fadd_rn(a.y, x.y), __fadd_rn(a.z, x.z), __fadd_rn(a.w, x.w));
+            }
+            dst[q] = x;
+        }
+    }
 }
 
 template <int B1, int B2, bool kVec>
 __global__ void __launch_bounds__(kThreads)
     qsgd_ts_merge_kernel(const __grid_constant__ RecordSet set, int W, float *__restrict__ out, int64_t n)
 {
+    __shared__ __align__(16) float s_vals[kWarpsPerBlock][kChunk];
     const int64_t off2 = sub_words(n, B1) + 3; // payload of the fine sub-record
     const float step1 = __fdiv_rn(f32_from_bits(set.rec[0][0]), (float)Levels<B1>::s);
     const float step2 = __fdiv_rn(f32_from_bits(set.rec[0][off2 - 3]), (float)Levels<B2>::s);
@@ -213,38 +342,51 @@ __global__ void __launch_bounds__(kThreads)
     const float bias1 = 8388608.0f + (float)(W << (B1 - 1));
     const float bias2 = 8388608.0f + (float)(W << (B2 - 1));
     const int64_t nwords1 = (n * B1 + 31) >> 5, nwords2 = (n * B2 + 31) >> 5;
-    const int64_t spans = (n + kSpan - 1) / kSpan;
-    for (int64_t sp = (int64_t)blockIdx.x * kThreads + threadIdx.x; sp < spans;
-         sp += (int64_t)gridDim.x * kThreads) {
-        uint32_t s1[kSpan], s2[kSpan];
-        span_sums<B1>(set, W, 3, sp, nwords1, s1);
-        span_sums<B2>(set, W, off2, sp, nwords2, s2);
-        float v[kSpan];
+    const int lane = threadIdx.x & (kWarp - 1);
+    float *sv = s_vals[threadIdx.x >> 5];
+    const float4 *sv4 = reinterpret_cast<const float4 *>(sv);
+    const int64_t chunks = (n + kChunk - 1) / kChunk;
+    for (int64_t ch = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5); ch < chunks;
+         ch += (int64_t)gridDim.x * kWarpsPerBlock) {
+        chunk_part<B1, false>(set, W, 3, ch, nwords1, lane, step1, bias1, sv);
+        __syncwarp();
+        chunk_part<B2, true>(set, W, off2, ch, nwords2, lane, step2, bias2, sv);
+        __syncwarp();
 #pragma unroll
-        for (int e = 0; e < kSpan; ++e) {
-            const float a = __fmul_rn(__fsub_rn(__uint_as_float(0x4B000000u | s1[e]), bias1), step1);
-            const float b = __fmul_rn(__fsub_rn(__uint_as_float(0x4B000000u | s2[e]), bias2), step2);
-            v[e] = __fadd_rn(a, b);
-        }
-        const int64_t e0 = sp * kSpan;
-        if (kVec && e0 + kSpan <= n) {
-            st_stream_f8(out + e0, v);
-            st_stream_f8(out + e0 + 8, v + 8);
-        } else {
+        for (int j = 0; j < kChunk / 4 / kWarp; ++j) {
+            const int q = j * kWarp + lane; // group of 4 within the chunk
+            const int64_t gi = ch * (kChunk / 4) + q;
+            const float4 x = sv4[q];
+            if (kVec && gi < (n >> 2)) {
+                st_stream_f4(out + 4 * gi, x);
+            } else {
+                const float xx[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-            for (int e = 0; e < kSpan; ++e)
-                if (e0 + e < n)
-                    st_stream_f1(out + e0 + e, v[e]);
+                for (int e = 0; e < 4; ++e)
+                    if (4 * gi + e < n)
+                        st_stream_f1(out + 4 * gi + e, xx[e]);
+            }
         }
+        __syncwarp();
     }
 }
 
 int bits_slot(int bits) { return bits == 2 ? 0 : (bits == 4 ? 1 : (bits == 8 ? 2 : -1)); }
 
 std::atomic<int> occ_tq[3][3][2][64];
+std::atomic<int> occ_tw[3][3][64];
+#ifndef QGA_TS_LANE_WORDS
+#define QGA_TS_LANE_WORDS 1
+#endif
 std::atomic<int> occ_tm[3][3][2][64];
 
-constexpr int kTsQuantizeWaves = 8, kTsMergeWaves = 8;
+#ifndef QGA_TS_MERGE_WAVES
+#define QGA_TS_MERGE_WAVES 8
+#endif
+#ifndef QGA_TS_QUANTIZE_WAVES
+#define QGA_TS_QUANTIZE_WAVES 8
+#endif
+constexpr int kTsQuantizeWaves = QGA_TS_QUANTIZE_WAVES, kTsMergeWaves = QGA_TS_MERGE_WAVES;
 
 template <int B1, int B2>
 void launch_quantize(const float *grad, uint32_t *compr, int64_t n, uint64_t seed, const float *M,
@@ -255,7 +397,13 @@ void launch_quantize(const float *grad, uint32_t *compr, int64_t n, uint64_t see
     const int64_t tiles = (groups + kTileGroups - 1) / kTileGroups;
     const int64_t blocks = (tiles + kWarpsPerBlock - 1) / kWarpsPerBlock;
     auto &occ = occ_tq[bits_slot(B1)][bits_slot(B2)];
-    if (aligned(grad, 16)) {
+    if (QGA_TS_LANE_WORDS && aligned(grad, 32)) {
+        auto k = qsgd_ts_quantize_words_kernel<B1, B2>;
+        const int64_t runs = (n + 16 * kWarp - 1) / (16 * kWarp);
+        k<<<grid_for((runs + kWarpsPerBlock - 1) / kWarpsPerBlock, resident_blocks(k, kThreads, occ_tw[bits_slot(B1)][bits_slot(B2)]),
+                     kTsQuantizeWaves),
+            kThreads, 0, stream>>>(grad, compr, n, k0, k1, M);
+    } else if (aligned(grad, 16)) {
         auto k = qsgd_ts_quantize_kernel<B1, B2, true>;
         k<<<grid_for(blocks, resident_blocks(k, kThreads, occ[0]), kTsQuantizeWaves), kThreads, 0,
             stream>>>(grad, compr, n, k0, k1, M);
@@ -269,10 +417,10 @@ void launch_quantize(const float *grad, uint32_t *compr, int64_t n, uint64_t see
 template <int B1, int B2>
 void launch_merge(const RecordSet &set, int W, float *out, int64_t n, cudaStream_t stream)
 {
-    const int64_t spans = (n + kSpan - 1) / kSpan;
-    const int64_t blocks = (spans + kThreads - 1) / kThreads;
+    const int64_t chunks = (n + kChunk - 1) / kChunk;
+    const int64_t blocks = (chunks + kWarpsPerBlock - 1) / kWarpsPerBlock;
     auto &occ = occ_tm[bits_slot(B1)][bits_slot(B2)];
-    if (aligned(out, 32)) {
+    if (aligned(out, 16)) {
         auto k = qsgd_ts_merge_kernel<B1, B2, true>;
         k<<<grid_for(blocks, resident_blocks(k, kThreads, occ[0]), kTsMergeWaves), kThreads, 0,
             stream>>>(set, W, out, n);
