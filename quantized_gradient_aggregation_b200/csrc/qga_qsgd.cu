@@ -247,8 +247,8 @@ __global__ void __launch_bounds__(kThreads)
 }
 
 // ----------------------------------------------------------------- merge ----
-// Integer sum of the W workers' levels a whole record word at a time (Swar,
-// swar_add_word in qga_qsgd_level.cuh).  A thread owns whole words: word l of
+// Integer sum of the W workers' levels a whole record word at a time
+// (LevelSum in qga_qsgd_level.cuh).  A thread owns whole words: word l of
 // each 32-word block of its warp (for b = 2, also word 32 + l, loaded
 // together for more bytes in flight), and stores its 32/b outputs as 128-bit
 // (b = 8) or 256-bit rows.
@@ -257,15 +257,15 @@ template <int B> constexpr int kMergeSlotsFor = B == 2 ? 2 : 1; // words per thr
 // Outputs of one record word from its lane sums: element e sits in field
 // kFields - 1 - e (counted from the least significant).
 template <int B, bool kVec>
-__device__ __forceinline__ void merge_store_word(const uint32_t (&acc)[Swar<B>::kRegs], int64_t kw,
-                                                 float offset, float step, float *__restrict__ out,
-                                                 int64_t n)
+__device__ __forceinline__ void merge_store_word(LevelSum<B> &acc, int64_t kw, float offset, float step,
+                                                 float *__restrict__ out, int64_t n)
 {
-    using S = Swar<B>;
+    using S = LevelSum<B>;
+    acc.finish();
     float v[S::kFields];
 #pragma unroll
     for (int e = 0; e < S::kFields; ++e)
-        v[e] = __fmul_rn(__fsub_rn(__uint_as_float(0x4B000000u | swar_field_sum<B>(acc, e)), offset), step);
+        v[e] = __fmul_rn(__fsub_rn(__uint_as_float(0x4B000000u | acc.field_sum(e)), offset), step);
     const int64_t e0 = kw * S::kFields;
     if (kVec && e0 + S::kFields <= n) {
         if (S::kFields == 4)
@@ -287,8 +287,8 @@ __global__ void __launch_bounds__(kThreads)
     qsgd_merge_kernel(const __grid_constant__ RecordSet set, int W, float *__restrict__ out,
                       int64_t n)
 {
-    using S = Swar<B>;
     constexpr int kBatch = 8;
+    static_assert(kBatch <= LevelSum<B>::kBatchMax, "a batch fits the narrow lanes");
     __shared__ const uint32_t *s_payload[QGA_MAX_WORKERS];
     if (threadIdx.x < W)
         s_payload[threadIdx.x] = set.rec[threadIdx.x] + 3;
@@ -300,7 +300,7 @@ __global__ void __launch_bounds__(kThreads)
     const int64_t stride = (int64_t)gridDim.x * kThreads;
     if constexpr (kMergeSlotsFor<B> == 1) {
         for (int64_t kw = (int64_t)blockIdx.x * kThreads + threadIdx.x; kw < nwords; kw += stride) {
-            uint32_t acc[S::kRegs] = {};
+            LevelSum<B> acc;
             for (int wb = 0; wb < W; wb += kBatch) {
                 uint32_t words[kBatch];
 #pragma unroll
@@ -310,8 +310,9 @@ __global__ void __launch_bounds__(kThreads)
                 for (int i = 0; i < kBatch; ++i) {
                     if (wb + i >= W) // warp-uniform
                         break;
-                    swar_add_word<B>(acc, words[i]);
+                    acc.add(words[i]);
                 }
+                acc.end_batch();
             }
             merge_store_word<B, kVec>(acc, kw, offset, step, out, n);
         }
@@ -323,7 +324,7 @@ __global__ void __launch_bounds__(kThreads)
         for (int64_t sl = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5; sl < nslices;
              sl += stride >> 5) {
             const int64_t k0 = sl * (2 * kWarp) + lane, k1 = k0 + kWarp;
-            uint32_t acc0[S::kRegs] = {}, acc1[S::kRegs] = {};
+            LevelSum<B> acc0, acc1;
             for (int wb = 0; wb < W; wb += kBatch) {
                 uint32_t w0[kBatch], w1[kBatch];
 #pragma unroll
@@ -335,9 +336,11 @@ __global__ void __launch_bounds__(kThreads)
                 for (int i = 0; i < kBatch; ++i) {
                     if (wb + i >= W) // warp-uniform
                         break;
-                    swar_add_word<B>(acc0, w0[i]);
-                    swar_add_word<B>(acc1, w1[i]);
+                    acc0.add(w0[i]);
+                    acc1.add(w1[i]);
                 }
+                acc0.end_batch();
+                acc1.end_batch();
             }
             if (k0 < nwords)
                 merge_store_word<B, kVec>(acc0, k0, offset, step, out, n);

@@ -187,41 +187,88 @@ __device__ __forceinline__ uint32_t signed_code(uint32_t L, float g)
 // ------------------------------------------------- integer sum of levels --
 // The merges add the W workers' levels a whole record word at a time.  XOR
 // with the sign bit of every b-bit field turns a two's-complement level q
-// into q + 2^(b-1) in [0, 2^b); masking every fourth (b = 2, 4) or every
-// other (b = 8) field spreads the biased fields into 8-bit (b = 2) or 16-bit
-// lanes of 32-bit registers, where one integer add sums a lane group over a
-// worker without carries crossing lanes (at most 64 workers: 64 * 3 < 2^8,
-// 64 * 255 < 2^16).  At the end each lane's sum, minus W * 2^(b-1), is the
-// exact integer level sum; it is below 2^23, so adding it to the bits of
-// 2^23 and subtracting 2^23 + W 2^(b-1) in binary32 converts it exactly.
-template <int B> struct Swar {
-    static constexpr int kFields = 32 / B;          // elements per word
-    static constexpr int kLaneBits = B == 2 ? 8 : 16;
-    static constexpr int kLanesPerReg = 32 / kLaneBits;
-    static constexpr int kRegs = kFields / kLanesPerReg;
-    static constexpr uint32_t kSign = B == 2 ? 0xAAAAAAAAu : (B == 4 ? 0x88888888u : 0x80808080u);
-    // fields j, j + kRegs, j + 2 kRegs, ... (counted from the least significant) -> register j
-    static constexpr uint32_t kMask = B == 2 ? 0x03030303u : (B == 4 ? 0x000F000Fu : 0x00FF00FFu);
+// into q + 2^(b-1) in [0, 2^b), and the biased fields are added in SIMD
+// lanes of registers wide enough that no add carries into the neighbouring
+// lane (at most 64 workers):
+//   b = 2: every fourth field in the 8-bit lanes of 4 registers (64 * 3 < 2^8);
+//   b = 4: the even and odd fields in the 8-bit lanes of 2 registers, which
+//          hold up to 17 words (17 * 15 < 2^8) and are widened into the
+//          16-bit lanes of 4 registers after every batch of words;
+//   b = 8: the even and odd fields in the 16-bit lanes of 2 registers
+//          (64 * 255 < 2^16).
+// A field's final sum, minus W 2^(b-1), is the exact integer level sum; it is
+// below 2^23, so adding it to the bits of 2^23 and subtracting 2^23 + W
+// 2^(b-1) in binary32 converts it exactly.
+//   add(word) for each worker's word, end_batch() after every batch of at
+//   most kBatchMax words, finish() at the end; field_sum(e) is the biased
+//   sum of element e of the word (element 0 = most significant field).
+template <int B> struct LevelSum;
+
+template <> struct LevelSum<2> {
+    static constexpr int kFields = 16, kBatchMax = 64;
+    static constexpr uint32_t kSign = 0xAAAAAAAAu;
+    uint32_t w[4] = {0u, 0u, 0u, 0u}; // register j: fields j, j + 4, j + 8, j + 12
+    __device__ __forceinline__ void add(uint32_t word)
+    {
+        const uint32_t x = word ^ kSign;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            w[j] += (x >> (2 * j)) & 0x03030303u;
+    }
+    __device__ __forceinline__ void end_batch() {}
+    __device__ __forceinline__ void finish() {}
+    __device__ __forceinline__ uint32_t field_sum(int e) const
+    {
+        const int f = kFields - 1 - e; // field counted from the least significant
+        return (w[f & 3] >> (8 * (f >> 2))) & 0xFFu;
+    }
 };
 
-template <int B>
-__device__ __forceinline__ void swar_add_word(uint32_t (&acc)[Swar<B>::kRegs], uint32_t word)
-{
-    using S = Swar<B>;
-    const uint32_t biased = word ^ S::kSign;
-#pragma unroll
-    for (int j = 0; j < S::kRegs; ++j)
-        acc[j] += (biased >> (B * j)) & S::kMask;
-}
+template <> struct LevelSum<4> {
+    static constexpr int kFields = 8, kBatchMax = 17;
+    static constexpr uint32_t kSign = 0x88888888u;
+    uint32_t a = 0u, b = 0u;          // 8-bit lanes: fields 2i (a), 2i + 1 (b)
+    uint32_t w[4] = {0u, 0u, 0u, 0u}; // 16-bit lanes: bytes 0 / 2 and 1 / 3 of a, then of b
+    __device__ __forceinline__ void add(uint32_t word)
+    {
+        const uint32_t x = word ^ kSign;
+        a += x & 0x0F0F0F0Fu;
+        b += (x >> 4) & 0x0F0F0F0Fu;
+    }
+    __device__ __forceinline__ void end_batch()
+    {
+        w[0] += a & 0x00FF00FFu;
+        w[1] += (a >> 8) & 0x00FF00FFu;
+        w[2] += b & 0x00FF00FFu;
+        w[3] += (b >> 8) & 0x00FF00FFu;
+        a = b = 0u;
+    }
+    __device__ __forceinline__ void finish() { end_batch(); }
+    __device__ __forceinline__ uint32_t field_sum(int e) const
+    {
+        const int f = kFields - 1 - e;
+        const int i = f >> 1; // byte of a (f even) or b (f odd)
+        return (w[2 * (f & 1) + (i & 1)] >> (16 * (i >> 1))) & 0xFFFFu;
+    }
+};
 
-// The biased sum (level sum + W 2^(b-1)) of element e of the word, element
-// 0 being the most significant field.
-template <int B>
-__device__ __forceinline__ uint32_t swar_field_sum(const uint32_t (&acc)[Swar<B>::kRegs], int e)
-{
-    using S = Swar<B>;
-    const int f = S::kFields - 1 - e;
-    return (acc[f % S::kRegs] >> (S::kLaneBits * (f / S::kRegs))) & ((1u << S::kLaneBits) - 1u);
-}
+template <> struct LevelSum<8> {
+    static constexpr int kFields = 4, kBatchMax = 64;
+    static constexpr uint32_t kSign = 0x80808080u;
+    uint32_t w[2] = {0u, 0u}; // 16-bit lanes: bytes 0 / 2 and 1 / 3
+    __device__ __forceinline__ void add(uint32_t word)
+    {
+        const uint32_t x = word ^ kSign;
+        w[0] += x & 0x00FF00FFu;
+        w[1] += (x >> 8) & 0x00FF00FFu;
+    }
+    __device__ __forceinline__ void end_batch() {}
+    __device__ __forceinline__ void finish() {}
+    __device__ __forceinline__ uint32_t field_sum(int e) const
+    {
+        const int f = kFields - 1 - e;
+        return (w[f & 1] >> (16 * (f >> 1))) & 0xFFFFu;
+    }
+};
 
 } // namespace qga

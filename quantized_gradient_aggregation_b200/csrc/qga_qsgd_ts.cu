@@ -23,7 +23,7 @@
 // 4 elements, lane l groups l, l+32, l+64, l+96; one Philox block per group),
 // the fixed-point level of qga_qsgd_level.cuh with E = max(b1, b2) - 1 and
 // the scale picked per element, and two packed outputs.  Merge: each scale's
-// levels summed over the workers in SIMD lanes of registers (swar_add_word)
+// levels summed over the workers in SIMD lanes of registers (LevelSum)
 // in that sub-record's own coalesced layout, converted and scaled once, and
 // the two parts added in shared memory (see qsgd_ts_merge_kernel).
 
@@ -269,7 +269,7 @@ __global__ void __launch_bounds__(kThreads)
 // A warp owns chunks of 512 elements.  Each sub-record is summed in its own
 // coalesced layout: the chunk's 16 b words, lane l owning words l, 32 + l,
 // ... (b / 2 of them), the levels of all workers added in SIMD lanes of
-// registers (swar_add_word); each element's sum is converted exactly,
+// registers (LevelSum); each element's sum is converted exactly,
 // scaled once by that scale's step and written to the warp's 2 KB of shared
 // memory (the coarse part), or added there to the coarse part (the fine
 // part).  The 512 results then leave as coalesced 128-bit rows.
@@ -288,10 +288,11 @@ __device__ __forceinline__ void chunk_part(const RecordSet &set, int W, int64_t 
                                            int64_t nwords, int lane, float step, float bias,
                                            float *__restrict__ sv)
 {
-    using S = Swar<B>;
+    using S = LevelSum<B>;
     constexpr int kWords = B / 2;
     constexpr int kBatch = QGA_TS_MERGE_BATCH;
-    uint32_t acc[kWords][S::kRegs] = {};
+    static_assert(kBatch <= LevelSum<B>::kBatchMax, "a batch fits the narrow lanes");
+    LevelSum<B> acc[kWords];
     for (int wb = 0; wb < W; wb += kBatch) {
         uint32_t words[kBatch][kWords];
 #pragma unroll
@@ -308,15 +309,19 @@ __device__ __forceinline__ void chunk_part(const RecordSet &set, int W, int64_t 
                 break;
 #pragma unroll
             for (int c = 0; c < kWords; ++c)
-                swar_add_word<B>(acc[c], words[i][c]);
+                acc[c].add(words[i][c]);
         }
+#pragma unroll
+        for (int c = 0; c < kWords; ++c)
+            acc[c].end_batch();
     }
 #pragma unroll
     for (int c = 0; c < kWords; ++c) {
+        acc[c].finish();
         float v[S::kFields];
 #pragma unroll
         for (int e = 0; e < S::kFields; ++e)
-            v[e] = __fmul_rn(__fsub_rn(__uint_as_float(0x4B000000u | swar_field_sum<B>(acc[c], e)), bias), step);
+            v[e] = __fmul_rn(__fsub_rn(__uint_as_float(0x4B000000u | acc[c].field_sum(e)), bias), step);
         float4 *dst = reinterpret_cast<float4 *>(sv + (c * kWarp + lane) * S::kFields);
 #pragma unroll
         for (int q = 0; q < S::kFields / 4; ++q) {
