@@ -47,7 +47,9 @@ TS_PAIRS = ((4, 8), (2, 4))          # QSGD-MN-TS rows: (coarse bits, fine bits)
 # launch of the quantize kernel (profiles/quantize_2bit_kernel_fp32_vgg16.md),
 # keyed by the hash of the sources that kernel is compiled from; reported as
 # null once they have changed since the capture.
-MEASURED_TRAFFIC = {"f29bd18f50f18594": 11.871}   # 1.6425 GB per launch of n = 138,357,544
+# DRAM bytes per element of one quantize launch (ncu, n = 34,589,386), keyed by
+# the code hash of the kernel sources; scaled by elements to the full launch.
+MEASURED_TRAFFIC = {"6271b0663c9cedf3": 10.749}   # 1.487 GB per launch of n = 138,357,544
 QUANT_SOURCES = ("qga_common.cuh", "qga_2bit_tiles.cuh", "qga_2bit.cu")
 
 
