@@ -53,14 +53,32 @@ def up_to_date() -> bool:
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile every source to an object in parallel (one nvcc per file,
+    under _build/), then link the shared library."""
     if not force and up_to_date():
         return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-o", tmp, *sources()]
-    if verbose:
-        cmd.insert(1, "-Xptxas=-v")
-    subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
+    objdir = os.path.join(PKG, "_build")
+    os.makedirs(objdir, exist_ok=True)
+    compile_flags = [f for f in NVCC_FLAGS if f != "-shared"]
+    jobs = []
+    for src in sources():
+        obj = os.path.join(objdir, os.path.splitext(os.path.basename(src))[0] + f".{os.getpid()}.o")
+        cmd = [nvcc(), *compile_flags, "-I", INCLUDE, "-c", "-o", obj, src]
+        if verbose:
+            cmd.insert(1, "-Xptxas=-v")
+        jobs.append((obj, subprocess.Popen(cmd)))
+    failed = [obj for obj, p in jobs if p.wait() != 0]
+    objs = [obj for obj, _ in jobs]
+    try:
+        if failed:
+            raise subprocess.CalledProcessError(1, f"nvcc ({len(failed)} of {len(jobs)} sources failed)")
+        tmp = LIB + f".tmp{os.getpid()}"
+        subprocess.run([nvcc(), *NVCC_FLAGS, "-o", tmp, *objs], check=True)
+        os.replace(tmp, LIB)
+    finally:
+        for obj in objs:
+            if os.path.exists(obj):
+                os.remove(obj)
     return LIB
 
 

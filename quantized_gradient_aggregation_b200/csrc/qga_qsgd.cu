@@ -350,6 +350,59 @@ __global__ void __launch_bounds__(kThreads)
     }
 }
 
+// The merge for a worker count known at compile time (W <= 8, one batch of
+// the level sums): the W payload pointers come from the kernel's parameter
+// space, and the W words of each of the lane's slots are all loaded before
+// any is summed.  A warp takes kMergeWSlots x 32 consecutive words: slot s of
+// lane l is word 32 s + l.  Four resident blocks of 256 threads per SM (at
+// most 64 registers).  Measured at n = 2^27, W = 8, b = 2 / 4 / 8: 125.4 /
+// 169.9 / 252.3 us, against 148.8 / 199 / 285 us for the runtime-W kernel
+// above, whose payload pointers are read back from shared memory in every
+// iteration; one slot per lane took 124.6 / 210.8 / 255.3 us, and 6 or 8
+// blocks per SM 140 / 171-217 / 256-263 us.
+#ifndef QGA_QSGD_MERGE_W_SLOTS
+#define QGA_QSGD_MERGE_W_SLOTS 2
+#endif
+#ifndef QGA_QSGD_MERGE_W_MIN_BLOCKS
+#define QGA_QSGD_MERGE_W_MIN_BLOCKS 4
+#endif
+constexpr int kMergeWSlots = QGA_QSGD_MERGE_W_SLOTS;
+
+template <int B, bool kVec, int kW>
+__global__ void __launch_bounds__(kThreads, QGA_QSGD_MERGE_W_MIN_BLOCKS)
+    qsgd_merge_w_kernel(const __grid_constant__ RecordSet set, float *__restrict__ out, int64_t n)
+{
+    constexpr int kSlots = kMergeWSlots;
+    static_assert(kW >= 1 && kW <= LevelSum<B>::kBatchMax, "one batch fits the narrow lanes");
+    const float step = __fdiv_rn(f32_from_bits(set.rec[0][0]), (float)Levels<B>::s);
+    const float offset = 8388608.0f + (float)(kW << (B - 1));
+    const int64_t nwords = (n * B + 31) >> 5;
+    const int lane = threadIdx.x & (kWarp - 1);
+    const int64_t nslices = (nwords + kSlots * kWarp - 1) / (kSlots * kWarp);
+    for (int64_t sl = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5; sl < nslices;
+         sl += ((int64_t)gridDim.x * kThreads) >> 5) {
+        uint32_t wd[kSlots][kW];
+#pragma unroll
+        for (int s = 0; s < kSlots; ++s) {
+            const int64_t k = (sl * kSlots + s) * kWarp + lane;
+#pragma unroll
+            for (int i = 0; i < kW; ++i)
+                wd[s][i] = k < nwords ? ld_stream_u32(set.rec[i] + 3 + k) : 0u;
+        }
+#pragma unroll
+        for (int s = 0; s < kSlots; ++s) {
+            const int64_t k = (sl * kSlots + s) * kWarp + lane;
+            LevelSum<B> acc;
+#pragma unroll
+            for (int i = 0; i < kW; ++i)
+                acc.add(wd[s][i]);
+            acc.end_batch();
+            if (k < nwords)
+                merge_store_word<B, kVec>(acc, k, offset, step, out, n);
+        }
+    }
+}
+
 std::atomic<int> occ_max[64];
 std::atomic<int> occ_q[3][2][64];
 std::atomic<int> occ_qw[3][64];
@@ -357,6 +410,7 @@ std::atomic<int> occ_qw[3][64];
 #define QGA_QSGD_LANE_WORDS 1
 #endif
 std::atomic<int> occ_m[3][2][64];
+std::atomic<int> occ_mw[3][2][9][64]; // [bits][vec][W][device]
 
 int bits_slot(int bits) { return bits == 2 ? 0 : (bits == 4 ? 1 : (bits == 8 ? 2 : -1)); }
 
@@ -370,6 +424,10 @@ int bits_slot(int bits) { return bits == 2 ? 0 : (bits == 4 ? 1 : (bits == 8 ? 2
 #endif
 constexpr int kQsgdQuantizeWaves = QGA_QSGD_QUANTIZE_WAVES;
 template <int B> constexpr int kQsgdMergeWaves = B == 8 ? 1 : 16;
+#ifndef QGA_QSGD_MERGE_W_WAVES
+#define QGA_QSGD_MERGE_W_WAVES 16
+#endif
+constexpr int kQsgdMergeWWaves = QGA_QSGD_MERGE_W_WAVES;
 
 template <int B>
 unsigned merge_grid(int64_t n, int resident)
@@ -409,10 +467,43 @@ void launch_quantize(const float *grad, uint32_t *compr, int64_t n, uint64_t see
     }
 }
 
+template <int B, bool kVec, int kW>
+void launch_merge_w(const RecordSet &set, float *out, int64_t n, cudaStream_t stream)
+{
+    auto k = qsgd_merge_w_kernel<B, kVec, kW>;
+    const int64_t nwords = (n * B + 31) >> 5;
+    const int64_t per_block = (int64_t)kThreads * kMergeWSlots;
+    k<<<grid_for((nwords + per_block - 1) / per_block, resident_blocks(k, kThreads, occ_mw[bits_slot(B)][kVec][kW]),
+                 kQsgdMergeWWaves),
+        kThreads, 0, stream>>>(set, out, n);
+}
+
+template <int B, bool kVec>
+void launch_merge_w(const RecordSet &set, int W, float *out, int64_t n, cudaStream_t stream)
+{
+    switch (W) {
+    case 1: launch_merge_w<B, kVec, 1>(set, out, n, stream); break;
+    case 2: launch_merge_w<B, kVec, 2>(set, out, n, stream); break;
+    case 3: launch_merge_w<B, kVec, 3>(set, out, n, stream); break;
+    case 4: launch_merge_w<B, kVec, 4>(set, out, n, stream); break;
+    case 5: launch_merge_w<B, kVec, 5>(set, out, n, stream); break;
+    case 6: launch_merge_w<B, kVec, 6>(set, out, n, stream); break;
+    case 7: launch_merge_w<B, kVec, 7>(set, out, n, stream); break;
+    default: launch_merge_w<B, kVec, 8>(set, out, n, stream); break;
+    }
+}
+
 template <int B>
 void launch_merge(const RecordSet &set, int W, float *out, int64_t n, cudaStream_t stream)
 {
     const int s = bits_slot(B);
+    if (W <= 8) {
+        if (aligned(out, 32))
+            launch_merge_w<B, true>(set, W, out, n, stream);
+        else
+            launch_merge_w<B, false>(set, W, out, n, stream);
+        return;
+    }
     if (aligned(out, 32)) {
         auto k = qsgd_merge_kernel<B, true>;
         k<<<merge_grid<B>(n, resident_blocks(k, kThreads, occ_m[s][0])), kThreads, 0, stream>>>(

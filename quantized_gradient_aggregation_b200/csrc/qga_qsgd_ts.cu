@@ -283,15 +283,17 @@ constexpr int kChunk = 512;
 #ifndef QGA_TS_MERGE_BATCH
 #define QGA_TS_MERGE_BATCH 4
 #endif
-template <int B, bool kAdd>
+template <int B, bool kAdd, int kW>
 __device__ __forceinline__ void chunk_part(const RecordSet &set, int W, int64_t payload_off, int64_t chunk,
                                            int64_t nwords, int lane, float step, float bias,
                                            float *__restrict__ sv)
 {
     using S = LevelSum<B>;
     constexpr int kWords = B / 2;
-    constexpr int kBatch = QGA_TS_MERGE_BATCH;
+    constexpr int kBatch = kW > 0 ? kW : QGA_TS_MERGE_BATCH;
     static_assert(kBatch <= LevelSum<B>::kBatchMax, "a batch fits the narrow lanes");
+    if (kW > 0)
+        W = kW;
     LevelSum<B> acc[kWords];
     for (int wb = 0; wb < W; wb += kBatch) {
         uint32_t words[kBatch][kWords];
@@ -335,10 +337,12 @@ __device__ __forceinline__ void chunk_part(const RecordSet &set, int W, int64_t 
     }
 }
 
-template <int B1, int B2, bool kVec>
+template <int B1, int B2, bool kVec, int kW>
 __global__ void __launch_bounds__(kThreads)
     qsgd_ts_merge_kernel(const __grid_constant__ RecordSet set, int W, float *__restrict__ out, int64_t n)
 {
+    if (kW > 0)
+        W = kW;
     __shared__ __align__(16) float s_vals[kWarpsPerBlock][kChunk];
     const int64_t off2 = sub_words(n, B1) + 3; // payload of the fine sub-record
     const float step1 = __fdiv_rn(f32_from_bits(set.rec[0][0]), (float)Levels<B1>::s);
@@ -353,9 +357,9 @@ __global__ void __launch_bounds__(kThreads)
     const int64_t chunks = (n + kChunk - 1) / kChunk;
     for (int64_t ch = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5); ch < chunks;
          ch += (int64_t)gridDim.x * kWarpsPerBlock) {
-        chunk_part<B1, false>(set, W, 3, ch, nwords1, lane, step1, bias1, sv);
+        chunk_part<B1, false, kW>(set, W, 3, ch, nwords1, lane, step1, bias1, sv);
         __syncwarp();
-        chunk_part<B2, true>(set, W, off2, ch, nwords2, lane, step2, bias2, sv);
+        chunk_part<B2, true, kW>(set, W, off2, ch, nwords2, lane, step2, bias2, sv);
         __syncwarp();
 #pragma unroll
         for (int j = 0; j < kChunk / 4 / kWarp; ++j) {
@@ -419,18 +423,45 @@ void launch_quantize(const float *grad, uint32_t *compr, int64_t n, uint64_t see
     }
 }
 
+// W <= 8 with an aligned output: the worker count as a template argument
+// (all W workers' words of a part loaded at once, payload pointers from the
+// parameter space).  Measured at n = 2^27, W = 8: (4, 8) 354 us, (2, 4) 226
+// us, (8, 2) 324 us, against 433 / 258 / 439 us with the runtime count.
+std::atomic<int> occ_tmw[3][3][9][64]; // [b1][b2][W][device]
+
+template <int B1, int B2, int kW>
+void launch_merge_w(const RecordSet &set, float *out, int64_t n, int64_t blocks, cudaStream_t stream)
+{
+    auto k = qsgd_ts_merge_kernel<B1, B2, true, kW>;
+    k<<<grid_for(blocks, resident_blocks(k, kThreads, occ_tmw[bits_slot(B1)][bits_slot(B2)][kW]), kTsMergeWaves),
+        kThreads, 0, stream>>>(set, kW, out, n);
+}
+
 template <int B1, int B2>
 void launch_merge(const RecordSet &set, int W, float *out, int64_t n, cudaStream_t stream)
 {
     const int64_t chunks = (n + kChunk - 1) / kChunk;
     const int64_t blocks = (chunks + kWarpsPerBlock - 1) / kWarpsPerBlock;
     auto &occ = occ_tm[bits_slot(B1)][bits_slot(B2)];
+    if (W <= 8 && aligned(out, 16)) {
+        switch (W) {
+        case 1: launch_merge_w<B1, B2, 1>(set, out, n, blocks, stream); break;
+        case 2: launch_merge_w<B1, B2, 2>(set, out, n, blocks, stream); break;
+        case 3: launch_merge_w<B1, B2, 3>(set, out, n, blocks, stream); break;
+        case 4: launch_merge_w<B1, B2, 4>(set, out, n, blocks, stream); break;
+        case 5: launch_merge_w<B1, B2, 5>(set, out, n, blocks, stream); break;
+        case 6: launch_merge_w<B1, B2, 6>(set, out, n, blocks, stream); break;
+        case 7: launch_merge_w<B1, B2, 7>(set, out, n, blocks, stream); break;
+        default: launch_merge_w<B1, B2, 8>(set, out, n, blocks, stream); break;
+        }
+        return;
+    }
     if (aligned(out, 16)) {
-        auto k = qsgd_ts_merge_kernel<B1, B2, true>;
+        auto k = qsgd_ts_merge_kernel<B1, B2, true, 0>;
         k<<<grid_for(blocks, resident_blocks(k, kThreads, occ[0]), kTsMergeWaves), kThreads, 0,
             stream>>>(set, W, out, n);
     } else {
-        auto k = qsgd_ts_merge_kernel<B1, B2, false>;
+        auto k = qsgd_ts_merge_kernel<B1, B2, false, 0>;
         k<<<grid_for(blocks, resident_blocks(k, kThreads, occ[1]), kTsMergeWaves), kThreads, 0,
             stream>>>(set, W, out, n);
     }

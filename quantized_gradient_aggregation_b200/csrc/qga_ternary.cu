@@ -309,14 +309,41 @@ __device__ __forceinline__ void add_trits(uint32_t v, uint32_t weight, uint32_t 
 
 // Words per lane of a table-merge tile (build-time setting; the default is
 // the measured best): lane l owns words l, 32 + l, ... and loads all of them,
-// of every worker, before using any.
+// of every worker, before using any.  With QGA_TERNARY_TABLE_PREFETCH the
+// words of the warp's next tile are loaded before the current tile is
+// decoded and stored, so that they are in flight meanwhile.  Measured at
+// n = 138M, W = 8: 2 slots with the next tile in flight 142.0 us; 2 slots
+// loaded just before use 148.9 us; 1 slot 158.7 us, with the next tile in
+// flight and 4 blocks per SM 145.7 us.
 #ifndef QGA_TERNARY_TABLE_SLOTS
 #define QGA_TERNARY_TABLE_SLOTS 2
 #endif
+#ifndef QGA_TERNARY_TABLE_PREFETCH
+#define QGA_TERNARY_TABLE_PREFETCH 1
+#endif
+#ifdef QGA_TERNARY_TABLE_MIN_BLOCKS
+#define QGA_TERNARY_TABLE_BOUNDS __launch_bounds__(kThreads, QGA_TERNARY_TABLE_MIN_BLOCKS)
+#else
+#define QGA_TERNARY_TABLE_BOUNDS __launch_bounds__(kThreads)
+#endif
 constexpr int kTernarySlots = QGA_TERNARY_TABLE_SLOTS;
+constexpr bool kTernaryPrefetch = QGA_TERNARY_TABLE_PREFETCH != 0;
+
+template <int kW>
+__device__ __forceinline__ void load_ternary_tile(const RecordSet &set, int64_t t, int64_t nwords, int lane,
+                                                  uint32_t (&words)[kTernarySlots][kW])
+{
+#pragma unroll
+    for (int sl = 0; sl < kTernarySlots; ++sl) {
+        const int64_t w = (t * kTernarySlots + sl) * kWarp + lane;
+#pragma unroll
+        for (int k = 0; k < kW; ++k)
+            words[sl][k] = w < nwords ? ld_stream_u32(set.rec[k] + 3 + w) : 0u;
+    }
+}
 
 template <bool kVec, int kW>
-__global__ void __launch_bounds__(kThreads)
+__global__ void QGA_TERNARY_TABLE_BOUNDS
     merge_ternary_table_kernel(const __grid_constant__ RecordSet set, float *__restrict__ out, int64_t n)
 {
     __shared__ float s_neg[kW], s_pos[kW];
@@ -327,21 +354,29 @@ __global__ void __launch_bounds__(kThreads)
         s_neg[threadIdx.x] = f32_from_bits(r[0]);
         s_pos[threadIdx.x] = f32_from_bits(r[1]);
     }
-    __syncthreads();
-    build_sum_table<kW>(s_sum, [&](int w) { return s_neg[w]; }, [&](int w) { return s_pos[w]; });
     const char *tb = reinterpret_cast<const char *>(s_sum);
     float4 *stage = s_stage[threadIdx.x >> 5];
     const int lane = threadIdx.x & (kWarp - 1);
     const int64_t nwords = (n + 19) / 20;
     const int64_t tiles = (nwords + kWarp * kTernarySlots - 1) / (kWarp * kTernarySlots);
-    for (int64_t t = warp_id(); t < tiles; t += warp_stride()) {
-        uint32_t words[kTernarySlots][kW];
+    int64_t t = warp_id();
+    uint32_t words[kTernarySlots][kW];
+    if (t < tiles) // the first tile's words are in flight while the table is built
+        load_ternary_tile<kW>(set, t, nwords, lane, words);
+    __syncthreads();
+    build_sum_table<kW>(s_sum, [&](int w) { return s_neg[w]; }, [&](int w) { return s_pos[w]; });
+    for (; t < tiles; t += warp_stride()) {
+        const int64_t tn = t + warp_stride();
+        uint32_t next[kTernarySlots][kW];
+        if (kTernaryPrefetch) {
+            if (tn < tiles)
+                load_ternary_tile<kW>(set, tn, nwords, lane, next);
+            else
 #pragma unroll
-        for (int sl = 0; sl < kTernarySlots; ++sl) {
-            const int64_t w = (t * kTernarySlots + sl) * kWarp + lane;
+                for (int sl = 0; sl < kTernarySlots; ++sl)
 #pragma unroll
-            for (int k = 0; k < kW; ++k)
-                words[sl][k] = w < nwords ? ld_stream_u32(set.rec[k] + 3 + w) : 0u;
+                    for (int k = 0; k < kW; ++k)
+                        next[sl][k] = 0u;
         }
 #pragma unroll
         for (int sl = 0; sl < kTernarySlots; ++sl) {
@@ -374,6 +409,15 @@ __global__ void __launch_bounds__(kThreads)
                 store_group<kVec>(out, n, g0 + q, stage[q]);
             }
             __syncwarp();
+        }
+        if (kTernaryPrefetch) {
+#pragma unroll
+            for (int sl = 0; sl < kTernarySlots; ++sl)
+#pragma unroll
+                for (int k = 0; k < kW; ++k)
+                    words[sl][k] = next[sl][k];
+        } else if (tn < tiles) {
+            load_ternary_tile<kW>(set, tn, nwords, lane, words);
         }
     }
 }

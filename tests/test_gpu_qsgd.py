@@ -95,7 +95,7 @@ def test_quantize_misaligned_and_special(b):
 
 
 @pytest.mark.parametrize("b", BITS)
-@pytest.mark.parametrize("W", [1, 2, 8, 64])
+@pytest.mark.parametrize("W", [1, 2, 3, 5, 7, 8, 9, 64])
 @pytest.mark.parametrize("n", [1, 17, 513, 65_537])
 def test_merge(b, W, n):
     q = qga()
@@ -118,6 +118,29 @@ def test_merge(b, W, n):
     got = f32(out)
     np.testing.assert_allclose(got, want, rtol=AGG_RTOL, atol=AGG_ATOL)
     assert same_bits_f32(got, want), first_diff(got, want)
+
+
+@pytest.mark.parametrize("b", BITS)
+@pytest.mark.parametrize("W", [1, 2, 3, 4, 5, 6, 7, 8, 9, 17, 64])
+def test_merge_random_records(b, W):
+    """Arbitrary bit patterns as records (every b-bit field value, -2^(b-1)
+    included, which no quantize writes) merge as the oracle merges them, for
+    every worker count of the compile-time kernels and beyond; n ragged and
+    the output misaligned for one worker count."""
+    q = qga()
+    n = 4099 + 16 * W
+    rng = np.random.default_rng(100 * b + W)
+    words = q.qga_qsgd_words(n, b)
+    recs = []
+    for w in range(W):
+        r = rng.integers(0, 1 << 32, words, dtype=np.uint64).astype(np.uint32)
+        r[0] = np.float32(0.75).view(np.uint32)
+        r[1], r[2] = np.float32(b).view(np.uint32), np.float32(n).view(np.uint32)
+        recs.append(r)
+    out = offset_view(n, torch.float32, 1 if W == 5 else 0, fill=float("nan"))
+    q.qga_qsgd_mn_dequant_accumulate([torch.from_numpy(r.view(np.int32)).to(DEV) for r in recs], out, b)
+    want = oracle.qsgd_mn_dequant_accumulate(recs, n, b)
+    assert same_bits_f32(f32(out), want), first_diff(f32(out), want)
 
 
 def _levels_of_word(word, b):

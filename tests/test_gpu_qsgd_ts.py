@@ -92,7 +92,7 @@ def test_quantize_boundary_misaligned_and_special(b1, b2):
 
 
 @pytest.mark.parametrize("b1,b2", PAIRS)
-@pytest.mark.parametrize("W", [1, 3, 8, 64])
+@pytest.mark.parametrize("W", [1, 2, 3, 5, 8, 9, 64])
 @pytest.mark.parametrize("n", [1, 17, 513, 65_537])
 def test_merge(b1, b2, W, n):
     q = qga()
@@ -107,7 +107,8 @@ def test_merge(b1, b2, W, n):
         assert np.array_equal(u32(c), want_c), w
         recs.append(c)
         want_recs.append(want_c)
-    out = offset_view(n, torch.float32, n % 3, fill=float("nan"))
+    # odd worker counts write an aligned output, even ones a misaligned one
+    out = offset_view(n, torch.float32, 0 if W % 2 else 1 + n % 3, fill=float("nan"))
     q.qga_qsgd_mnts_dequant_accumulate(recs, out, b1, b2)
     want = oracle.qsgd_mnts_dequant_accumulate(want_recs, n, b1, b2)
     got = f32(out)
@@ -116,12 +117,14 @@ def test_merge(b1, b2, W, n):
 
 
 @pytest.mark.parametrize("b1,b2", [(2, 4), (4, 8), (8, 2)])
-def test_merge_random_records(b1, b2):
+@pytest.mark.parametrize("W", [1, 2, 3, 4, 5, 6, 7, 8, 9, 17])
+def test_merge_random_records(b1, b2, W):
     """Arbitrary bit patterns in both sub-records (every level value, both
-    signs, on both scales at once) merge as the oracle merges them."""
+    signs, on both scales at once) merge as the oracle merges them, for every
+    worker count of the compile-time kernels and beyond."""
     q = qga()
-    n, W = 4099, 8
-    rng = np.random.default_rng(b1 * 16 + b2)
+    n = 4099 + 32 * W
+    rng = np.random.default_rng(b1 * 16 + b2 + 1000 * W)
     words = q.qga_qsgd_mnts_words(n, b1, b2)
     w1 = 3 + -(-(n * b1) // 32)
     recs = []
