@@ -43,13 +43,12 @@ QUANT_BYTES_PER_ELEM = 12.25        # read g 4 + read r 4 + write r 4 + write co
 FALLBACK_HBM_GBS = 6650.0
 TS_PAIRS = ((4, 8), (2, 4))          # QSGD-MN-TS rows: (coarse bits, fine bits)
 
-# dram__bytes_read.sum + dram__bytes_write.sum per element of one full-size
-# launch of the quantize kernel (profiles/quantize_2bit_kernel_fp32_vgg16.md),
-# keyed by the hash of the sources that kernel is compiled from; reported as
-# null once they have changed since the capture.
-# DRAM bytes per element of one quantize launch (ncu, n = 34,589,386), keyed by
-# the code hash of the kernel sources; scaled by elements to the full launch.
-MEASURED_TRAFFIC = {"6271b0663c9cedf3": 10.749}   # 1.487 GB per launch of n = 138,357,544
+# dram__bytes_read.sum + dram__bytes_write.sum per element of one launch of
+# the quantize kernel, captured at n = 34,589,386
+# (profiles/quantize_2bit_kernel_fp32_vgg16.md) and scaled by elements to the
+# full launch; keyed by the code hash of the sources that kernel is compiled
+# from, and reported as null once they have changed since the capture.
+MEASURED_TRAFFIC = {"c1bfd2432f8b046e": 10.735}   # 1.485 GB per launch of n = 138,357,544
 QUANT_SOURCES = ("qga_common.cuh", "qga_2bit_tiles.cuh", "qga_2bit.cu")
 
 
