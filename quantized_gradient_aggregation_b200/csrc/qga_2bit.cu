@@ -182,10 +182,18 @@ std::atomic<int> occ_tab[2][9][64]; // [vec][kW][device]: W <= 8
 // 256); dequantize 109 / 97 / 96 / 101 us at 1 / 8 / 16 / 32; merge (W = 8)
 // 180 / 174 / 176 / 181 us at 1 / 8 / 16 / 32.
 constexpr int kQuantizeWaves = 32, kDequantizeWaves = 16, kMergeWaves = 8;
-#ifndef QGA_TABLE_MERGE_WAVES
-#define QGA_TABLE_MERGE_WAVES 1
+// The table merge by worker count: every block builds the 3^W-entry table
+// once, so small tables take many waves and large ones one persistent wave.
+// Measured at n = 138M (us at 1 / 2 / 4 / 8 / 16 waves): W = 1 108 / 103 /
+// 97 / 95 / 93, W = 2 115 / 112 / 104 / 99 / 98, W = 3 121 / 118 / 110 / 105
+// / 103, W = 4 127 / 123 / 115 / 111 / 112, W = 5 120 / 119 / 119 / 119 /
+// 121, W = 6 126 / 127 / 127 / 132 / 138, W = 7 131 / 132 / 133 / 136 / 144,
+// W = 8 142 / 142 / 144 / 152 / 169.
+#ifdef QGA_TABLE_MERGE_WAVES
+constexpr int table_merge_waves(int) { return QGA_TABLE_MERGE_WAVES; }
+#else
+constexpr int table_merge_waves(int w) { return w <= 3 ? 16 : (w == 4 ? 8 : (w == 5 ? 2 : 1)); }
 #endif
-constexpr int kTableMergeWaves = QGA_TABLE_MERGE_WAVES;
 
 unsigned tiles_grid(int64_t n, int resident, int64_t elems_per_warp, int waves)
 {
@@ -199,7 +207,7 @@ void launch_merge_k(const RecordSet &set, int W, float *out, int64_t n, cudaStre
     if constexpr (kW > 0) {
         auto k = merge_2bit_table_kernel<kVec, kW>;
         k<<<tiles_grid(n, resident_blocks(k, kThreads, occ_tab[kVec][kW]), kMergeSliceElems,
-                       kTableMergeWaves),
+                       table_merge_waves(kW)),
             kThreads, 0, stream>>>(set, out, n);
     } else {
         auto k = dequant_accumulate_2bit_kernel<kVec, 0>;

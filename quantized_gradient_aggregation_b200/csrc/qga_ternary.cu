@@ -428,10 +428,16 @@ std::atomic<int> occ_tq[2][64], occ_td[2][2][9][64]; // td: [vec][merge][kW]
 // 243 / 240 us at 1 / 8 / 16 / 32 / 128 waves; merge (W = 8) 206 / 199 / 206
 // / 224 us at 1 / 8 / 16 / 32.
 constexpr int kTernaryQuantizeWaves = 32, kTernaryDecodeWaves = 8;
-#ifndef QGA_TERNARY_TABLE_WAVES
-#define QGA_TERNARY_TABLE_WAVES 1
+// The table merge by worker count (the table is rebuilt by every block):
+// measured at n = 138M (us at 1 / 4 / 8 / 16 waves): W = 1 106 / 95 / 93 /
+// 91, W = 2 112 / 100 / 97 / 96, W = 3 117 / 105 / 101 / 99, W = 4 123 / 110
+// / 107 / 111, W = 5 128 / 114 / 110 / 115, W = 6 134 / 119 / 119 / 134,
+// W = 7 139 / 125 / 131 / 152, W = 8 142 / 147 / 158 / 187.
+#ifdef QGA_TERNARY_TABLE_WAVES
+constexpr int ternary_table_waves(int) { return QGA_TERNARY_TABLE_WAVES; }
+#else
+constexpr int ternary_table_waves(int w) { return w <= 3 ? 16 : (w <= 5 ? 8 : (w <= 7 ? 4 : 1)); }
 #endif
-constexpr int kTernaryTableWaves = QGA_TERNARY_TABLE_WAVES;
 
 unsigned warps_grid(int64_t warp_items, int resident, int waves)
 {
@@ -446,7 +452,7 @@ void launch_decode_k(const RecordSet &set, int W, float *out, int64_t n, cudaStr
         auto k = merge_ternary_table_kernel<kVec, kW>;
         const int64_t table_tiles = ((n + 19) / 20 + kWarp * kTernarySlots - 1) / (kWarp * kTernarySlots);
         k<<<warps_grid(table_tiles, resident_blocks(k, kThreads, occ_td[kVec][kMerge][kW]),
-                       kTernaryTableWaves),
+                       ternary_table_waves(kW)),
             kThreads, 0, stream>>>(set, out, n);
     } else {
         auto k = decode_ternary_kernel<kVec, kMerge, kW>;
