@@ -283,7 +283,21 @@ constexpr int kChunk = 512;
 #ifndef QGA_TS_MERGE_BATCH
 #define QGA_TS_MERGE_BATCH 4
 #endif
-template <int B, bool kAdd, int kW>
+
+// Shared-memory slot of group g (4 elements) of a chunk.  A lane writes the
+// kFields / 4 consecutive groups of its word, so at b = 2 (b = 4) the lanes
+// of a quarter-warp are 4 (2) groups apart and meet in the same banks.  With
+// kSwizzle the XOR with bits 3..5 of g spreads them over all 8 slots of a
+// 128-byte row for b = 2, 4 and 8 alike, and keeps the 8 consecutive groups
+// of a coalesced output row in one row of 8 slots.  Measured at 2^27
+// (plain / swizzled, us): (2, 4) W = 1 172 / 123, W = 2 184 / 142, W = 4
+// 181 / 172, W = 6 204 / 211, W = 8 226 / 234; (4, 8) W = 1 128 / 142, W = 4
+// 231 / 222, W = 8 354 / 356.  So the swizzle is used where a part has b = 2
+// and the worker count is at most 4.
+template <bool kSwizzle>
+__device__ __forceinline__ int group_slot(int g) { return kSwizzle ? g ^ ((g >> 3) & 7) : g; }
+
+template <int B, bool kAdd, int kW, bool kSwizzle>
 __device__ __forceinline__ void chunk_part(const RecordSet &set, int W, int64_t payload_off, int64_t chunk,
                                            int64_t nwords, int lane, float step, float bias,
                                            float *__restrict__ sv)
@@ -324,15 +338,16 @@ __device__ __forceinline__ void chunk_part(const RecordSet &set, int W, int64_t 
 #pragma unroll
         for (int e = 0; e < S::kFields; ++e)
             v[e] = __fmul_rn(__fsub_rn(__uint_as_float(0x4B000000u | acc[c].field_sum(e)), bias), step);
-        float4 *dst = reinterpret_cast<float4 *>(sv + (c * kWarp + lane) * S::kFields);
+        float4 *sv4 = reinterpret_cast<float4 *>(sv);
 #pragma unroll
         for (int q = 0; q < S::kFields / 4; ++q) {
+            const int slot = group_slot<kSwizzle>((c * kWarp + lane) * (S::kFields / 4) + q);
             float4 x = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
             if (kAdd) {
-                const float4 a = dst[q];
+                const float4 a = sv4[slot];
                 x = make_float4(__fadd_rn(a.x, x.x), __fadd_rn(a.y, x.y), __fadd_rn(a.z, x.z), __fadd_rn(a.w, x.w));
             }
-            dst[q] = x;
+            sv4[slot] = x;
         }
     }
 }
@@ -343,6 +358,7 @@ __global__ void __launch_bounds__(kThreads)
 {
     if (kW > 0)
         W = kW;
+    constexpr bool kSwizzle = (B1 == 2 || B2 == 2) && kW >= 1 && kW <= 4;
     __shared__ __align__(16) float s_vals[kWarpsPerBlock][kChunk];
     const int64_t off2 = sub_words(n, B1) + 3; // payload of the fine sub-record
     const float step1 = __fdiv_rn(f32_from_bits(set.rec[0][0]), (float)Levels<B1>::s);
@@ -357,15 +373,15 @@ __global__ void __launch_bounds__(kThreads)
     const int64_t chunks = (n + kChunk - 1) / kChunk;
     for (int64_t ch = (int64_t)blockIdx.x * kWarpsPerBlock + (threadIdx.x >> 5); ch < chunks;
          ch += (int64_t)gridDim.x * kWarpsPerBlock) {
-        chunk_part<B1, false, kW>(set, W, 3, ch, nwords1, lane, step1, bias1, sv);
+        chunk_part<B1, false, kW, kSwizzle>(set, W, 3, ch, nwords1, lane, step1, bias1, sv);
         __syncwarp();
-        chunk_part<B2, true, kW>(set, W, off2, ch, nwords2, lane, step2, bias2, sv);
+        chunk_part<B2, true, kW, kSwizzle>(set, W, off2, ch, nwords2, lane, step2, bias2, sv);
         __syncwarp();
 #pragma unroll
         for (int j = 0; j < kChunk / 4 / kWarp; ++j) {
             const int q = j * kWarp + lane; // group of 4 within the chunk
             const int64_t gi = ch * (kChunk / 4) + q;
-            const float4 x = sv4[q];
+            const float4 x = sv4[group_slot<kSwizzle>(q)];
             if (kVec && gi < (n >> 2)) {
                 st_stream_f4(out + 4 * gi, x);
             } else {
