@@ -282,6 +282,12 @@ __device__ __forceinline__ void merge_store_word(LevelSum<B> &acc, int64_t kw, f
     }
 }
 
+// Any worker count (used for W > 8): batches of 8 workers, the payload
+// pointers read from the kernel's parameter space.  Measured at n = 2^27,
+// b = 4, W = 9 / 16 / 32: 212 / 279 / 467 us, against 230 / 312 / 533 us
+// with the pointers read back from shared memory in every iteration (b = 2
+// and 8 unchanged).  Two slots per lane for every b, 4 blocks per SM and a
+// separate full-batch path measured far slower (b = 8, W = 32: 1448 us).
 template <int B, bool kVec>
 __global__ void __launch_bounds__(kThreads)
     qsgd_merge_kernel(const __grid_constant__ RecordSet set, int W, float *__restrict__ out,
@@ -289,10 +295,6 @@ __global__ void __launch_bounds__(kThreads)
 {
     constexpr int kBatch = 8;
     static_assert(kBatch <= LevelSum<B>::kBatchMax, "a batch fits the narrow lanes");
-    __shared__ const uint32_t *s_payload[QGA_MAX_WORKERS];
-    if (threadIdx.x < W)
-        s_payload[threadIdx.x] = set.rec[threadIdx.x] + 3;
-    __syncthreads();
     const float step = __fdiv_rn(f32_from_bits(set.rec[0][0]), (float)Levels<B>::s);
     // 2^23 + W 2^(b-1): the magic-number conversion's offset and the bias
     const float offset = 8388608.0f + (float)(W << (B - 1));
@@ -305,7 +307,7 @@ __global__ void __launch_bounds__(kThreads)
                 uint32_t words[kBatch];
 #pragma unroll
                 for (int i = 0; i < kBatch; ++i)
-                    words[i] = wb + i < W ? ld_stream_u32(s_payload[wb + i] + kw) : 0u;
+                    words[i] = wb + i < W ? ld_stream_u32(set.rec[wb + i] + 3 + kw) : 0u;
 #pragma unroll
                 for (int i = 0; i < kBatch; ++i) {
                     if (wb + i >= W) // warp-uniform
@@ -329,8 +331,8 @@ __global__ void __launch_bounds__(kThreads)
                 uint32_t w0[kBatch], w1[kBatch];
 #pragma unroll
                 for (int i = 0; i < kBatch; ++i) {
-                    w0[i] = (wb + i < W && k0 < nwords) ? ld_stream_u32(s_payload[wb + i] + k0) : 0u;
-                    w1[i] = (wb + i < W && k1 < nwords) ? ld_stream_u32(s_payload[wb + i] + k1) : 0u;
+                    w0[i] = (wb + i < W && k0 < nwords) ? ld_stream_u32(set.rec[wb + i] + 3 + k0) : 0u;
+                    w1[i] = (wb + i < W && k1 < nwords) ? ld_stream_u32(set.rec[wb + i] + 3 + k1) : 0u;
                 }
 #pragma unroll
                 for (int i = 0; i < kBatch; ++i) {
@@ -357,7 +359,7 @@ __global__ void __launch_bounds__(kThreads)
 // lane l is word 32 s + l.  Four resident blocks of 256 threads per SM (at
 // most 64 registers).  Measured at n = 2^27, W = 8, b = 2 / 4 / 8: 125.4 /
 // 169.9 / 252.3 us, against 148.8 / 199 / 285 us for the runtime-W kernel
-// above, whose payload pointers are read back from shared memory in every
+// above when it read the payload pointers back from shared memory in every
 // iteration; one slot per lane took 124.6 / 210.8 / 255.3 us, and 6 or 8
 // blocks per SM 140 / 171-217 / 256-263 us.
 #ifndef QGA_QSGD_MERGE_W_SLOTS
