@@ -12,8 +12,9 @@
 // best for each kernel (see grid_for).  Nothing is filled
 // or cleared by a separate launch: the quantize kernel writes every payload
 // word (including the zero tail codes) and its block 0 writes the header.
-// The merge's occupancy and words per lane are build-time settings
-// (QGA_MERGE_MIN_BLOCKS, QGA_MERGE_SLOTS); the defaults are the measured best.
+// The merges are built for W <= 8 from a table of all 3^W sums, and for
+// W > 8 from the table of the first 8 workers' sums continued by per-worker
+// adds.
 
 #include "qga_2bit_tiles.cuh"
 
@@ -83,45 +84,6 @@ struct RecordSet {
     const uint32_t *rec[QGA_MAX_WORKERS];
 };
 
-// kW > 0: compiled for exactly kW workers (record pointers and loop bounds
-// are constants); kW == 0: any W up to QGA_MAX_WORKERS.
-#ifndef QGA_MERGE_MIN_BLOCKS
-#define QGA_MERGE_MIN_BLOCKS 4
-#endif
-
-template <bool kVec, int kW>
-__global__ void __launch_bounds__(kThreads, QGA_MERGE_MIN_BLOCKS)
-    dequant_accumulate_2bit_kernel(const __grid_constant__ RecordSet set, int W,
-                                   float *__restrict__ out, int64_t n)
-{
-    __shared__ const uint32_t *s_payload[QGA_MAX_WORKERS];
-    __shared__ float s_neg[QGA_MAX_WORKERS], s_pos[QGA_MAX_WORKERS];
-    __shared__ float2 s_table[QGA_MAX_WORKERS][16];
-    __shared__ float4 s_stage[kWarpsPerBlock][kStagePerWarp];
-    if (threadIdx.x < W) {
-        const uint32_t *r = set.rec[threadIdx.x];
-        s_payload[threadIdx.x] = r + 3;
-        s_neg[threadIdx.x] = f32_from_bits(r[0]);
-        s_pos[threadIdx.x] = f32_from_bits(r[1]);
-    }
-    __syncthreads();
-    for (int i = threadIdx.x; i < W * 16; i += kThreads)
-        s_table[i >> 4][i & 15] = pair_entry(i & 15, s_neg[i >> 4], s_pos[i >> 4]);
-    __syncthreads();
-    const int lane = threadIdx.x & (kWarp - 1);
-    const int64_t slices = (n + kSliceElems - 1) / kSliceElems;
-    for (int64_t sl = first_tile(); sl < slices; sl += tile_stride()) {
-        if (kW > 0)
-            dequant_accumulate_2bit_slice<kVec, kW>(
-                W, [&](int w) { return set.rec[w] + 3; }, [&](int w) { return s_neg[w]; },
-                [&](int w) { return s_pos[w]; }, s_table, out, n, sl, lane, s_stage[threadIdx.x >> 5]);
-        else
-            dequant_accumulate_2bit_slice<kVec, 0>(
-                W, [&](int w) { return s_payload[w]; }, [&](int w) { return s_neg[w]; },
-                [&](int w) { return s_pos[w]; }, s_table, out, n, sl, lane, s_stage[threadIdx.x >> 5]);
-    }
-}
-
 // W <= 8: the merge through the table of all 3^W sums (build_sum_table,
 // merge_2bit_table_store): one table index and one shared-memory load per
 // element instead of W decodes and adds.  A lane owns one word of each of
@@ -171,9 +133,150 @@ __global__ void __launch_bounds__(kThreads, 4)
     }
 }
 
+// W > 8: the table of the first 8 workers' 3^8 sums gives each element's
+// exact running sum after worker 7 (one table load), and workers 8 .. W-1
+// are then added in order by the per-worker decode (pair tables for even
+// workers, bit masks and predicated adds for odd ones), so the result is
+// the definition's sum in worker order, bit for bit.  A lane owns one word
+// of each 32-word slice.  The 3^8 table (26,244 B) and the W - 8 pair
+// tables sit in dynamic shared memory.
+// Measured at n = 138M (us, W = 9 / 16 / 32): the first 8 words loaded just
+// before use 198 / 297 / 611 at 8 waves; the next slice's first 8 words in
+// flight 181 / 285 / 595 at 1 wave and 199 / 293 / 566 at 8 waves, against
+// 251 / 355 / 651 for the per-worker decode of all W workers.
+#ifndef QGA_PREFIX_MERGE_PREFETCH
+#define QGA_PREFIX_MERGE_PREFETCH 1
+#endif
+#ifdef QGA_PREFIX_MERGE_WAVES
+inline int prefix_merge_waves(int) { return QGA_PREFIX_MERGE_WAVES; }
+#else
+inline int prefix_merge_waves(int w) { return w <= 16 ? 1 : 8; }
+#endif
+constexpr int kPrefixWorkers = 8;
+constexpr int kPrefixTableBytes = Pow3<kPrefixWorkers>::value * 4;
+
+inline int hybrid_smem_bytes(int W)
+{
+    return kPrefixTableBytes + 4 /* pad to 8 */ + (W - kPrefixWorkers) * 16 * 8 + 2 * W * 4;
+}
+
+template <bool kVec>
+__global__ void __launch_bounds__(kThreads)
+    merge_2bit_prefix_table_kernel(const __grid_constant__ RecordSet set, int W, float *__restrict__ out,
+                                   int64_t n)
+{
+    extern __shared__ __align__(16) unsigned char s_dyn[];
+    float *s_sum = reinterpret_cast<float *>(s_dyn);
+    float2(*s_pair)[16] = reinterpret_cast<float2(*)[16]>(s_dyn + kPrefixTableBytes + 4);
+    float *s_neg = reinterpret_cast<float *>(s_dyn + kPrefixTableBytes + 4 + (W - kPrefixWorkers) * 128);
+    float *s_pos = s_neg + W;
+    __shared__ float4 s_stage[kWarpsPerBlock][kWarp * 4];
+    for (int w = threadIdx.x; w < W; w += kThreads) {
+        const uint32_t *r = set.rec[w];
+        s_neg[w] = f32_from_bits(r[0]);
+        s_pos[w] = f32_from_bits(r[1]);
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < (W - kPrefixWorkers) * 16; i += kThreads)
+        s_pair[i >> 4][i & 15] = pair_entry(i & 15, s_neg[kPrefixWorkers + (i >> 4)], s_pos[kPrefixWorkers + (i >> 4)]);
+    build_sum_table<kPrefixWorkers>(s_sum, [&](int w) { return s_neg[w]; }, [&](int w) { return s_pos[w]; });
+    const char *tb = reinterpret_cast<const char *>(s_sum);
+    const int lane = threadIdx.x & (kWarp - 1);
+    const int f = (lane >> 1) & 3;
+    float4 *stage = s_stage[threadIdx.x >> 5];
+    const int64_t nwords = (n + 15) >> 4;
+    const int64_t slices = (nwords + kWarp - 1) / kWarp;
+#if QGA_PREFIX_MERGE_PREFETCH
+    uint32_t wd[kTableMaxWorkers];
+    {
+        const int64_t k0 = first_tile() * kWarp + lane;
+#pragma unroll
+        for (int w = 0; w < kPrefixWorkers; ++w)
+            wd[w] = (first_tile() < slices && k0 < nwords) ? ld_stream_u32(set.rec[w] + 3 + k0) : 0u;
+    }
+#endif
+    for (int64_t sl = first_tile(); sl < slices; sl += tile_stride()) {
+        const int64_t k = sl * kWarp + lane;
+        const bool ok = k < nwords;
+        float2 acc[8];
+        {
+#if QGA_PREFIX_MERGE_PREFETCH
+            uint32_t nx[kTableMaxWorkers];
+            const int64_t kn = (sl + tile_stride()) * kWarp + lane;
+#pragma unroll
+            for (int w = 0; w < kPrefixWorkers; ++w)
+                nx[w] = (sl + tile_stride() < slices && kn < nwords) ? ld_stream_u32(set.rec[w] + 3 + kn) : 0u;
+#else
+            uint32_t wd[kTableMaxWorkers];
+#pragma unroll
+            for (int w = 0; w < kPrefixWorkers; ++w)
+                wd[w] = ok ? ld_stream_u32(set.rec[w] + 3 + k) : 0u;
+#endif
+            uint32_t off[16];
+            sum_table_offsets<kPrefixWorkers>(wd, off);
+#pragma unroll
+            for (int p = 0; p < 8; ++p)
+                acc[p] = make_float2(*reinterpret_cast<const float *>(tb + off[2 * p]),
+                                     *reinterpret_cast<const float *>(tb + off[2 * p + 1]));
+#if QGA_PREFIX_MERGE_PREFETCH
+#pragma unroll
+            for (int w = 0; w < kPrefixWorkers; ++w)
+                wd[w] = nx[w];
+#endif
+        }
+        for (int wb = kPrefixWorkers; wb < W; wb += kMergeBatch) {
+            uint32_t words[kMergeBatch];
+#pragma unroll
+            for (int i = 0; i < kMergeBatch; ++i)
+                words[i] = (ok && wb + i < W) ? ld_stream_u32(set.rec[wb + i] + 3 + k) : 0u;
+#pragma unroll
+            for (int i = 0; i < kMergeBatch; ++i) {
+                if (wb + i >= W) // warp-uniform
+                    break;
+                if ((i & 1) == 0) {
+                    const char *pt = reinterpret_cast<const char *>(s_pair[wb + i - kPrefixWorkers]);
+#pragma unroll
+                    for (int p = 0; p < 8; ++p) {
+                        // 4 code bits of elements 2p, 2p+1, times the 8-byte entry size
+                        const int sh = 25 - 4 * p;
+                        const uint32_t o = (sh >= 0 ? (words[i] >> sh) : (words[i] << (-sh))) & 0x78u;
+                        acc[p] = __fadd2_rn(acc[p], *reinterpret_cast<const float2 *>(pt + o));
+                    }
+                } else {
+                    const float neg = s_neg[wb + i], pos = s_pos[wb + i];
+                    const uint32_t lo = words[i] & 0x55555555u;
+                    const uint32_t hi = (words[i] >> 1) & 0x55555555u;
+                    const uint32_t is01 = lo & ~hi, is10 = hi & ~lo;
+#pragma unroll
+                    for (int p = 0; p < 16; ++p) {
+                        const uint32_t bit = 1u << (30 - 2 * p);
+                        float &a = (p & 1) ? acc[p >> 1].y : acc[p >> 1].x;
+                        if (is01 & bit)
+                            a = __fadd_rn(a, pos);
+                        if (is10 & bit)
+                            a = __fadd_rn(a, neg);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+            stage[lane * 4 + (c ^ f)] = make_float4(acc[2 * c].x, acc[2 * c].y, acc[2 * c + 1].x, acc[2 * c + 1].y);
+        __syncwarp();
+        const int64_t g0 = sl * kWarp * 4; // first group of this slice
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int q = j * kWarp + lane;
+            store_group<kVec>(out, n, g0 + q, stage[stage_slot(q >> 2, q & 3)]);
+        }
+        __syncwarp();
+    }
+}
+
 std::atomic<int> occ_q_f32_w[64], occ_q_f32_v[64], occ_q_f32_s[64], occ_q_bf16_v[64], occ_q_bf16_s[64];
 std::atomic<int> occ_dq_v[64], occ_dq_s[64];
 std::atomic<int> occ_acc[2][64];    // [vec][device]: W > 8
+std::atomic<bool> smem_attr_set[2][64];
 std::atomic<int> occ_tab[2][9][64]; // [vec][kW][device]: W <= 8
 
 // Grid waves (see grid_for), measured at n = 138M: quantize in group tiles
@@ -181,7 +284,7 @@ std::atomic<int> occ_tab[2][9][64]; // [vec][kW][device]: W <= 8
 // lane-owned words 252 / 243 us at 8 / 32 waves (2 words per lane: 253 /
 // 256); dequantize 109 / 97 / 96 / 101 us at 1 / 8 / 16 / 32; merge (W = 8)
 // 180 / 174 / 176 / 181 us at 1 / 8 / 16 / 32.
-constexpr int kQuantizeWaves = 32, kDequantizeWaves = 16, kMergeWaves = 8;
+constexpr int kQuantizeWaves = 32, kDequantizeWaves = 16;
 // The table merge by worker count: every block builds the 3^W-entry table
 // once, so small tables take many waves and large ones one persistent wave.
 // Measured at n = 138M (us at 1 / 2 / 4 / 8 / 16 waves): W = 1 108 / 103 /
@@ -210,9 +313,21 @@ void launch_merge_k(const RecordSet &set, int W, float *out, int64_t n, cudaStre
                        table_merge_waves(kW)),
             kThreads, 0, stream>>>(set, out, n);
     } else {
-        auto k = dequant_accumulate_2bit_kernel<kVec, 0>;
-        k<<<tiles_grid(n, resident_blocks(k, kThreads, occ_acc[kVec]), kSliceElems, kMergeWaves),
-            kThreads, 0, stream>>>(set, W, out, n);
+        // the prefix table needs more than the default 48 KB of shared memory:
+        // the attribute is set once per device, for the largest worker count
+        auto k = merge_2bit_prefix_table_kernel<kVec>;
+        const int smem = hybrid_smem_bytes(W);
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+            dev = 0;
+        if (!smem_attr_set[kVec][dev].load(std::memory_order_relaxed)) {
+            cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 hybrid_smem_bytes(QGA_MAX_WORKERS));
+            smem_attr_set[kVec][dev].store(true, std::memory_order_relaxed);
+        }
+        k<<<tiles_grid(n, resident_blocks(k, kThreads, occ_acc[kVec], hybrid_smem_bytes(QGA_MAX_WORKERS)),
+                       16 * kWarp, prefix_merge_waves(W)),
+            kThreads, smem, stream>>>(set, W, out, n);
     }
 }
 

@@ -112,7 +112,7 @@ int sm_count();
 // Blocks of `threads` threads that one SM keeps resident for `kernel`
 // (cached per kernel and device by the caller-provided slot).
 template <typename Kernel>
-int resident_blocks(Kernel kernel, int threads, std::atomic<int> *slots)
+int resident_blocks(Kernel kernel, int threads, std::atomic<int> *slots, size_t dynamic_smem = 0)
 {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
@@ -121,7 +121,7 @@ int resident_blocks(Kernel kernel, int threads, std::atomic<int> *slots)
     if (cached > 0)
         return cached;
     int blocks = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, kernel, threads, 0) != cudaSuccess ||
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, kernel, threads, dynamic_smem) != cudaSuccess ||
         blocks < 1)
         blocks = 1;
     slots[dev].store(blocks, std::memory_order_relaxed);

@@ -161,7 +161,7 @@ def test_dequantize(n, oo):
     assert same_bits_f32(f32(out), oracle.dequantize_2bit(words, n))
 
 
-@pytest.mark.parametrize("W", [1, 2, 3, 8, 9, 17, 64])
+@pytest.mark.parametrize("W", [1, 2, 3, 8, 9, 10, 17, 33, 64])
 @pytest.mark.parametrize("n", [1, 17, 513, 4097, 65_537])
 def test_dequant_accumulate(W, n):
     rng = np.random.default_rng(W * 1000 + n)
@@ -175,7 +175,7 @@ def test_dequant_accumulate(W, n):
     assert same_bits_f32(got, want), first_diff(got, want)
 
 
-@pytest.mark.parametrize("W", [1, 2, 5, 8, 9])
+@pytest.mark.parametrize("W", [1, 2, 5, 8, 9, 16])
 def test_dequant_accumulate_code_11_reads_as_zero(W):
     """Records holding the unused code 11 (never written by a quantize): it
     reads as +0 in the merge, for every worker count (the table merge clears
@@ -190,7 +190,7 @@ def test_dequant_accumulate_code_11_reads_as_zero(W):
     assert same_bits_f32(f32(out), want), first_diff(f32(out), want)
 
 
-@pytest.mark.parametrize("W", [2, 8])
+@pytest.mark.parametrize("W", [2, 8, 9, 16])
 def test_dequant_accumulate_shared_and_signed_zero_thresholds(W):
     """Thresholds shared by all workers, and -0 as a negative threshold
     (code 10 then adds -0, which leaves a +0 sum at +0)."""
