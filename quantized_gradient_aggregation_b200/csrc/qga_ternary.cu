@@ -176,100 +176,38 @@ struct RecordSet {
 #define QGA_TERNARY_TABLE_SHARE 1
 #endif
 
-// kMerge: sum of W records from +0 in worker order (bit for bit the 2-bit
-// merge's sums); otherwise W == 1 and each element is its code's value.
-// As in the 2-bit merge, even workers go through a per-worker pair table
-// (shared loads + paired adds) and odd workers through code masks and
-// predicated adds (skipping the exact +0 adds of code 00), so that neither
-// the integer pipe nor the load/store pipe saturates alone.
-// kW > 0: compiled for exactly kW workers (record pointers from the kernel
-// parameters and loop bounds are constants); kW == 0: any W.
-template <bool kVec, bool kMerge, int kW>
+// The dequantize of one dense record: a lane owns one word (20 elements),
+// turns its 4 bytes into 01 / 10 code masks through a 256-entry shared
+// table and writes each element's value; outputs leave through a stride-5
+// stage as coalesced 128-bit rows.
+template <bool kVec>
 __global__ void __launch_bounds__(kThreads)
-    decode_ternary_kernel(const __grid_constant__ RecordSet set, int W_runtime,
-                          float *__restrict__ out, int64_t n)
+    dequantize_ternary_kernel(const uint32_t *__restrict__ compr, float *__restrict__ out, int64_t n)
 {
-    const int W = kW > 0 ? kW : W_runtime;
     __shared__ uint16_t s_masks[256], s_codes[256];
-    __shared__ const uint32_t *s_payload[QGA_MAX_WORKERS];
-    __shared__ float s_neg[QGA_MAX_WORKERS], s_pos[QGA_MAX_WORKERS];
-    __shared__ float2 s_pair[kMerge ? QGA_MAX_WORKERS : 1][16];
     __shared__ float4 s_stage[kWarpsPerBlock][kWarp * 5];
     build_byte_tables(s_masks, s_codes);
-    if (threadIdx.x < W) {
-        const uint32_t *r = set.rec[threadIdx.x];
-        s_payload[threadIdx.x] = r + 3;
-        s_neg[threadIdx.x] = f32_from_bits(r[0]);
-        s_pos[threadIdx.x] = f32_from_bits(r[1]);
-    }
     __syncthreads();
-    if (kMerge)
-        for (int i = threadIdx.x; i < W * 16; i += kThreads)
-            s_pair[i >> 4][i & 15] = pair_entry(i & 15, s_neg[i >> 4], s_pos[i >> 4]);
-    __syncthreads();
+    const float neg = f32_from_bits(compr[0]), pos = f32_from_bits(compr[1]);
+    const uint32_t *payload = compr + 3;
     float4 *stage = s_stage[threadIdx.x >> 5];
     const int lane = threadIdx.x & (kWarp - 1);
     const int64_t nwords = (n + 19) / 20;
     const int64_t tiles = (nwords + kWarp - 1) / kWarp;
     for (int64_t t = warp_id(); t < tiles; t += warp_stride()) {
         const int64_t w = t * kWarp + lane;
-        const bool ok = w < nwords;
-        float2 acc[10];
+        const uint32_t word = w < nwords ? ld_stream_u32(payload + w) : 0u;
+        uint32_t is01, is10;
+        word_masks(s_masks, word, is01, is10);
+        float v[20];
 #pragma unroll
-        for (int q = 0; q < 10; ++q)
-            acc[q] = make_float2(0.0f, 0.0f);
-        constexpr int kBatch = 8;
-        for (int wb = 0; wb < W; wb += kBatch) {
-            uint32_t words[kBatch];
-#pragma unroll
-            for (int i = 0; i < kBatch; ++i)
-                words[i] = (ok && wb + i < W)
-                               ? ld_stream_u32((kW > 0 ? set.rec[wb + i] + 3 : s_payload[wb + i]) + w)
-                               : 0u;
-#pragma unroll
-            for (int i = 0; i < kBatch; ++i) {
-                if (wb + i >= W) // warp-uniform
-                    break;
-                const uint32_t word = words[i];
-                if (kMerge && (i % QGA_TERNARY_TABLE_PERIOD) < QGA_TERNARY_TABLE_SHARE) {
-                    // the 20 codes as a 40-bit string, element 0 in bits 39..38
-                    const uint32_t c0 = s_codes[word & 0xFFu], c1 = s_codes[(word >> 8) & 0xFFu];
-                    const uint32_t c2 = s_codes[(word >> 16) & 0xFFu], c3 = s_codes[word >> 24];
-                    const uint32_t hi = c0 >> 2;
-                    const uint32_t lo = (c0 << 30) | (c1 << 20) | (c2 << 10) | c3;
-                    const char *tb = reinterpret_cast<const char *>(s_pair[wb + i]);
-#pragma unroll
-                    for (int q = 0; q < 10; ++q) {
-                        // 4 code bits of elements 2q, 2q+1, times the 8-byte entry size
-                        const int sh = 36 - 4 * q;
-                        const uint32_t nib = sh >= 32 ? (hi >> (sh - 32)) : (lo >> sh);
-                        const uint32_t off = (nib & 0xFu) << 3;
-                        acc[q] = __fadd2_rn(acc[q], *reinterpret_cast<const float2 *>(tb + off));
-                    }
-                } else {
-                    const float neg = s_neg[wb + i], pos = s_pos[wb + i];
-                    uint32_t is01, is10;
-                    word_masks(s_masks, word, is01, is10);
-#pragma unroll
-                    for (int p = 0; p < 20; ++p) {
-                        const uint32_t bit = 1u << (19 - p);
-                        float &a = (p & 1) ? acc[p >> 1].y : acc[p >> 1].x;
-                        if (kMerge) {
-                            if (is01 & bit)
-                                a = __fadd_rn(a, pos);
-                            if (is10 & bit)
-                                a = __fadd_rn(a, neg);
-                        } else {
-                            a = (is01 & bit) ? pos : ((is10 & bit) ? neg : 0.0f);
-                        }
-                    }
-                }
-            }
+        for (int p = 0; p < 20; ++p) {
+            const uint32_t bit = 1u << (19 - p);
+            v[p] = (is01 & bit) ? pos : ((is10 & bit) ? neg : 0.0f);
         }
 #pragma unroll
         for (int c = 0; c < 5; ++c)
-            stage[5 * lane + c] = make_float4(acc[2 * c].x, acc[2 * c].y, acc[2 * c + 1].x,
-                                              acc[2 * c + 1].y);
+            stage[5 * lane + c] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
         __syncwarp();
 #pragma unroll
         for (int j = 0; j < 5; ++j) {
@@ -422,7 +360,124 @@ __global__ void QGA_TERNARY_TABLE_BOUNDS
     }
 }
 
+// W > 8: the first 8 workers' sum of each element from the 3^8 table (as in
+// merge_ternary_table_kernel), which is exactly the definition's running sum
+// after worker 7, then workers 8 .. W-1 added in order by the per-worker
+// decode (pair tables for even workers, code masks for odd ones).  The 3^8
+// table (26,244 B) sits in dynamic
+// shared memory.
+constexpr int kTernaryPrefix = 8;
+constexpr int kTernaryPrefixBytes = Pow3<kTernaryPrefix>::value * 4;
+
+template <bool kVec>
+__global__ void __launch_bounds__(kThreads)
+    merge_ternary_prefix_kernel(const __grid_constant__ RecordSet set, int W, float *__restrict__ out,
+                                int64_t n)
+{
+    extern __shared__ __align__(16) unsigned char s_dyn[];
+    float *s_sum = reinterpret_cast<float *>(s_dyn);
+    __shared__ uint16_t s_masks[256], s_codes[256];
+    __shared__ float s_neg[QGA_MAX_WORKERS], s_pos[QGA_MAX_WORKERS];
+    __shared__ float2 s_pair[QGA_MAX_WORKERS][16];
+    __shared__ float4 s_stage[kWarpsPerBlock][kWarp * 5];
+    build_byte_tables(s_masks, s_codes);
+    for (int w = threadIdx.x; w < W; w += kThreads) {
+        const uint32_t *r = set.rec[w];
+        s_neg[w] = f32_from_bits(r[0]);
+        s_pos[w] = f32_from_bits(r[1]);
+    }
+    __syncthreads();
+    for (int i = kTernaryPrefix * 16 + threadIdx.x; i < W * 16; i += kThreads)
+        s_pair[i >> 4][i & 15] = pair_entry(i & 15, s_neg[i >> 4], s_pos[i >> 4]);
+    build_sum_table<kTernaryPrefix>(s_sum, [&](int w) { return s_neg[w]; }, [&](int w) { return s_pos[w]; });
+    __syncthreads();
+    const char *tb = reinterpret_cast<const char *>(s_sum);
+    float4 *stage = s_stage[threadIdx.x >> 5];
+    const int lane = threadIdx.x & (kWarp - 1);
+    const int64_t nwords = (n + 19) / 20;
+    const int64_t tiles = (nwords + kWarp - 1) / kWarp;
+    for (int64_t t = warp_id(); t < tiles; t += warp_stride()) {
+        const int64_t w = t * kWarp + lane;
+        const bool ok = w < nwords;
+        float2 acc[10];
+        {
+            uint32_t ev[5] = {}, od[5] = {};
+            uint32_t weight = 4u;
+#pragma unroll
+            for (int k = 0; k < kTernaryPrefix; ++k) {
+                const uint32_t word = ok ? ld_stream_u32(set.rec[k] + 3 + w) : 0u;
+                add_trits(word & 0x00FF00FFu, weight, ev);
+                add_trits((word >> 8) & 0x00FF00FFu, weight, od);
+                weight *= 3u;
+            }
+            // byte b of the word holds elements 5b .. 5b + 4 (trit i = element 5b + i)
+            float v[20];
+#pragma unroll
+            for (int i = 0; i < 5; ++i) {
+                v[i] = *reinterpret_cast<const float *>(tb + (ev[i] & 0xFFFFu));
+                v[10 + i] = *reinterpret_cast<const float *>(tb + (ev[i] >> 16));
+                v[5 + i] = *reinterpret_cast<const float *>(tb + (od[i] & 0xFFFFu));
+                v[15 + i] = *reinterpret_cast<const float *>(tb + (od[i] >> 16));
+            }
+#pragma unroll
+            for (int q = 0; q < 10; ++q)
+                acc[q] = make_float2(v[2 * q], v[2 * q + 1]);
+        }
+        constexpr int kBatch = 8;
+        for (int wb = kTernaryPrefix; wb < W; wb += kBatch) {
+            uint32_t words[kBatch];
+#pragma unroll
+            for (int i = 0; i < kBatch; ++i)
+                words[i] = (ok && wb + i < W) ? ld_stream_u32(set.rec[wb + i] + 3 + w) : 0u;
+#pragma unroll
+            for (int i = 0; i < kBatch; ++i) {
+                if (wb + i >= W) // warp-uniform
+                    break;
+                const uint32_t word = words[i];
+                if ((i % QGA_TERNARY_TABLE_PERIOD) < QGA_TERNARY_TABLE_SHARE) {
+                    // the 20 codes as a 40-bit string, element 0 in bits 39..38
+                    const uint32_t c0 = s_codes[word & 0xFFu], c1 = s_codes[(word >> 8) & 0xFFu];
+                    const uint32_t c2 = s_codes[(word >> 16) & 0xFFu], c3 = s_codes[word >> 24];
+                    const uint32_t hi = c0 >> 2;
+                    const uint32_t lo = (c0 << 30) | (c1 << 20) | (c2 << 10) | c3;
+                    const char *pt = reinterpret_cast<const char *>(s_pair[wb + i]);
+#pragma unroll
+                    for (int q = 0; q < 10; ++q) {
+                        const int sh = 36 - 4 * q;
+                        const uint32_t nib = sh >= 32 ? (hi >> (sh - 32)) : (lo >> sh);
+                        acc[q] = __fadd2_rn(acc[q], *reinterpret_cast<const float2 *>(pt + ((nib & 0xFu) << 3)));
+                    }
+                } else {
+                    const float neg = s_neg[wb + i], pos = s_pos[wb + i];
+                    uint32_t is01, is10;
+                    word_masks(s_masks, word, is01, is10);
+#pragma unroll
+                    for (int p = 0; p < 20; ++p) {
+                        const uint32_t bit = 1u << (19 - p);
+                        float &a = (p & 1) ? acc[p >> 1].y : acc[p >> 1].x;
+                        if (is01 & bit)
+                            a = __fadd_rn(a, pos);
+                        if (is10 & bit)
+                            a = __fadd_rn(a, neg);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < 5; ++c)
+            stage[5 * lane + c] = make_float4(acc[2 * c].x, acc[2 * c].y, acc[2 * c + 1].x, acc[2 * c + 1].y);
+        __syncwarp();
+#pragma unroll
+        for (int j = 0; j < 5; ++j) {
+            const int q = j * kWarp + lane; // group of 4 within the tile
+            store_group<kVec>(out, n, t * (kWarp * 5) + q, stage[q]);
+        }
+        __syncwarp();
+    }
+}
+
 std::atomic<int> occ_tq[2][64], occ_td[2][2][9][64]; // td: [vec][merge][kW]
+std::atomic<bool> prefix_attr_set[2][64];
 
 // Grid waves (see grid_for), measured at n = 138M: quantize 287 / 253 / 247 /
 // 243 / 240 us at 1 / 8 / 16 / 32 / 128 waves; merge (W = 8) 206 / 199 / 206
@@ -454,10 +509,23 @@ void launch_decode_k(const RecordSet &set, int W, float *out, int64_t n, cudaStr
         k<<<warps_grid(table_tiles, resident_blocks(k, kThreads, occ_td[kVec][kMerge][kW]),
                        ternary_table_waves(kW)),
             kThreads, 0, stream>>>(set, out, n);
+    } else if constexpr (kMerge) {
+        // W > 8: the prefix table takes more than the default 48 KB of shared memory
+        auto k = merge_ternary_prefix_kernel<kVec>;
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+            dev = 0;
+        if (!prefix_attr_set[kVec][dev].load(std::memory_order_relaxed)) {
+            cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kTernaryPrefixBytes);
+            prefix_attr_set[kVec][dev].store(true, std::memory_order_relaxed);
+        }
+        k<<<warps_grid(tiles, resident_blocks(k, kThreads, occ_td[kVec][kMerge][0], kTernaryPrefixBytes),
+                       kTernaryDecodeWaves),
+            kThreads, kTernaryPrefixBytes, stream>>>(set, W, out, n);
     } else {
-        auto k = decode_ternary_kernel<kVec, kMerge, kW>;
-        k<<<warps_grid(tiles, resident_blocks(k, kThreads, occ_td[kVec][kMerge][kW]), kTernaryDecodeWaves),
-            kThreads, 0, stream>>>(set, W, out, n);
+        auto k = dequantize_ternary_kernel<kVec>;
+        k<<<warps_grid(tiles, resident_blocks(k, kThreads, occ_td[kVec][0][0]), kTernaryDecodeWaves),
+            kThreads, 0, stream>>>(set.rec[0], out, n);
     }
 }
 

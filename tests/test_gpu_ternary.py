@@ -99,7 +99,7 @@ def test_dequantize_ternary(n, oo):
     assert same_bits_f32(f32(out), oracle.dequantize_ternary(rec, n))
 
 
-@pytest.mark.parametrize("W", [1, 3, 8, 9, 17])
+@pytest.mark.parametrize("W", [1, 3, 8, 9, 17, 33, 64])
 @pytest.mark.parametrize("n", [21, 641, 65_537])
 def test_dequant_accumulate_ternary(W, n):
     rng = np.random.default_rng(W + n)
