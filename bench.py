@@ -48,7 +48,7 @@ TS_PAIRS = ((4, 8), (2, 4))          # QSGD-MN-TS rows: (coarse bits, fine bits)
 # (profiles/quantize_2bit_kernel_fp32_vgg16.md) and scaled by elements to the
 # full launch; keyed by the code hash of the sources that kernel is compiled
 # from, and reported as null once they have changed since the capture.
-MEASURED_TRAFFIC = {"c1bfd2432f8b046e": 10.735}   # 1.485 GB per launch of n = 138,357,544
+MEASURED_TRAFFIC = {"8903ee0898fe5645": 10.738}   # 1.486 GB per launch of n = 138,357,544
 QUANT_SOURCES = ("qga_common.cuh", "qga_2bit_tiles.cuh", "qga_2bit.cu")
 
 
