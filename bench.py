@@ -51,6 +51,30 @@ TS_PAIRS = ((4, 8), (2, 4))          # QSGD-MN-TS rows: (coarse bits, fine bits)
 MEASURED_TRAFFIC = {"8903ee0898fe5645": 10.738}   # 1.486 GB per launch of n = 138,357,544
 QUANT_SOURCES = ("qga_common.cuh", "qga_2bit_tiles.cuh", "qga_2bit.cu")
 
+# ALU-pipe thread instructions per element (ncu sm__inst_executed_pipe_alu.sum
+# x 32 / elements, captured at n = 2^25, profiles/row_kernels_quarter_size.md)
+# of the integer-bound QSGD quantizers, keyed by the code hash of their
+# sources; a row's "alu" object is null once the sources have changed.
+QSGD_SOURCES = ("qga_common.cuh", "qga_qsgd_level.cuh", "qga_qsgd.cu")
+TS_SOURCES = ("qga_common.cuh", "qga_qsgd_level.cuh", "qga_qsgd_ts.cu")
+MEASURED_ALU = {
+    "f0cac2ee0dafa582": {"b2": 12.78, "b4": 12.88, "b8": 13.58},
+    "cec14726e428f3f1": {"b4_8": 23.03, "b2_4": 21.50},
+}
+ALU_CLOCK_MHZ = 1965.0   # clocks.max.sm of the B200
+
+
+def alu_bound(instr_per_elem, elems, seconds, sms):
+    """The ALU-pipe roofline of an integer-bound kernel: one warp-instruction
+    every other cycle per SM sub-partition (4 per SM) at the maximum SM
+    clock; returns the bound's time and the fraction of it achieved."""
+    if instr_per_elem is None:
+        return None
+    per_s = sms * 4 * 0.5 * ALU_CLOCK_MHZ * 1e6   # warp-instructions per second
+    bound = elems * instr_per_elem / 32 / per_s
+    return {"alu_instr_per_elem": instr_per_elem, "bound_us": bound * 1e6, "frac": bound / seconds,
+            "clock_mhz": ALU_CLOCK_MHZ, "sms": sms}
+
 
 def parse_args():
     p = argparse.ArgumentParser()
@@ -613,6 +637,9 @@ def time_rows(dev, stream, peak, reps=20, scale=1, warmup=3):
     rows["qsgd_mn_max_w8"] = _row(t, nq * Wq, 4.0, peak, reps + warmup,
                                   workload=f"8 x {nq:,} fp32 (0.1% outliers of 50)")
     out = torch.empty(nq, device=dev)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    alu_q = MEASURED_ALU.get(csrc_hash(QSGD_SOURCES), {})
+    alu_ts = MEASURED_ALU.get(csrc_hash(TS_SOURCES), {})
     for b in wq.bits:
         cq = [torch.empty(q.qga_qsgd_words(nq, b), dtype=torch.int32, device=dev) for _ in range(Wq)]
 
@@ -624,7 +651,8 @@ def time_rows(dev, stream, peak, reps=20, scale=1, warmup=3):
             quant_q(k)
         t = _time_launches(stream, quant_q, reps, warmup)
         rows[f"qsgd_mn_quantize_b{b}"] = _row(t, nq, 4 + b / 8, peak, reps + warmup + Wq,
-                                              workload=f"{nq:,} fp32, b={b}")
+                                              workload=f"{nq:,} fp32, b={b}",
+                                              alu=alu_bound(alu_q.get(f"b{b}"), nq, t, sms))
         carr = (ctypes.c_void_p * Wq)(*[cc.data_ptr() for cc in cq])
         cp = ctypes.cast(carr, ctypes.POINTER(ctypes.c_void_p))
         t = _time_launches(stream, lambda: ok(L.qga_qsgd_mn_dequant_accumulate(
@@ -646,7 +674,8 @@ def time_rows(dev, stream, peak, reps=20, scale=1, warmup=3):
             quant_ts(k)
         t = _time_launches(stream, quant_ts, reps, warmup)
         rows[f"qsgd_mnts_quantize_b{b1}_{b2}"] = _row(t, nq, 4 + (b1 + b2) / 8, peak, reps + warmup + Wq,
-                                                      workload=f"{nq:,} fp32, b1={b1}, b2={b2}")
+                                                      workload=f"{nq:,} fp32, b1={b1}, b2={b2}",
+                                                      alu=alu_bound(alu_ts.get(f"b{b1}_{b2}"), nq, t, sms))
         carr = (ctypes.c_void_p * Wq)(*[cc.data_ptr() for cc in ct])
         cp = ctypes.cast(carr, ctypes.POINTER(ctypes.c_void_p))
         t = _time_launches(stream, lambda: ok(L.qga_qsgd_mnts_dequant_accumulate(

@@ -36,3 +36,20 @@ def test_workload_config_names_the_step():
     assert "quantize" in cfg["workload"] and "merge" in cfg["workload"]
     assert cfg["parallelism"].startswith("replicas x2")
     assert "L2" in cfg["l2"]
+
+
+def test_alu_bound_is_the_half_rate_alu_pipe_at_the_max_clock():
+    # 148 SMs x 4 sub-partitions x 0.5 warp-instructions per cycle at 1965 MHz
+    per_s = 148 * 4 * 0.5 * 1965e6
+    r = bench.alu_bound(12.0, 2**27, 200e-6, 148)
+    assert abs(r["bound_us"] - 2**27 * 12.0 / 32 / per_s * 1e6) < 1e-9
+    assert abs(r["frac"] - r["bound_us"] / 200.0) < 1e-12
+    assert bench.alu_bound(None, 2**27, 200e-6, 148) is None
+
+
+def test_measured_alu_rows_name_every_quantizer_of_the_bench():
+    for counts in bench.MEASURED_ALU.values():
+        assert all(v > 0 for v in counts.values())
+    keys = set().union(*bench.MEASURED_ALU.values())
+    assert {"b2", "b4", "b8"} <= keys
+    assert {f"b{b1}_{b2}" for b1, b2 in bench.TS_PAIRS} <= keys
