@@ -139,3 +139,67 @@ class BucketedCompressedAllGather:
         for b, work in enumerate(works):
             work.wait()  # the current stream waits for bucket b's records only
             self._merge(self.records(b), self.sizes[b], outs[b])
+
+
+class PeerMergeExchange:
+    """The exchange with the merge reading every rank's record where it lies.
+
+    Each rank quantizes into a record buffer of its own.  The buffers are
+    opened in every other rank by CUDA IPC (mappings of the owners' device
+    memory), so each rank's merge kernel loads all W records directly: the
+    peers' words cross NVLink / NVSwitch as plain loads inside the merge,
+    once, overlapped with its arithmetic and output stores, and no
+    all-gathered copy is written or read back.  The kernels are the
+    library's ordinary merges; a peer's buffer is just another record
+    pointer (plain loads only; nothing multicast).
+
+    Ordering across ranks is one host barrier per step: a rank synchronizes
+    its stream after its quantize, then waits for the group, then merges.
+    Record buffers alternate between two sets, so a rank overwrites set
+    s % 2 only at step s + 2, after the barrier of step s + 1, which every
+    rank reaches only after its merge of step s is complete.
+
+    ``close()`` releases the mappings of the peers' buffers (call it on
+    every rank before the group is destroyed).  Same arguments and formats
+    as ``CompressedAllGather``.
+    """
+
+    def __init__(self, n: int, neg_threshold: float, pos_threshold: float, group=None,
+                 fmt: str = "2bit", *, device=None):
+        from torch.multiprocessing.reductions import reduce_tensor
+        if fmt not in _FORMATS:
+            raise ValueError(f"format {fmt!r}: one of {sorted(_FORMATS)}")
+        self.n = int(n)
+        self.neg = float(neg_threshold)
+        self.pos = float(pos_threshold)
+        self.group = group
+        self.world = dist.get_world_size(group)
+        self.rank = dist.get_rank(group)
+        words_fn, self._quantize, self._merge = _FORMATS[fmt]
+        self.words = int(words_fn(self.n))
+        if device is None:
+            device = torch.device("cuda", torch.cuda.current_device())
+        self.local = [torch.zeros(self.words, dtype=torch.int32, device=device) for _ in range(2)]
+        torch.cuda.synchronize(device)
+        specs = [reduce_tensor(buf) for buf in self.local]
+        everyone = [None] * self.world
+        dist.all_gather_object(everyone, specs, group=self.group)
+        # records[k][r]: rank r's buffer of set k (this rank's own, or a mapping of a peer's)
+        self.records = [[self.local[k] if r == self.rank else everyone[r][k][0](*everyone[r][k][1])
+                         for r in range(self.world)] for k in range(2)]
+        self._step = 0
+
+    def step(self, grad: torch.Tensor, residual: torch.Tensor, out: torch.Tensor) -> None:
+        k = self._step & 1
+        self._quantize(grad, residual, self.local[k], self.neg, self.pos)
+        torch.cuda.current_stream(self.local[k].device).synchronize()
+        dist.barrier(group=self.group)  # every rank's record of this step is complete
+        self._merge(self.records[k], out)
+        self._step += 1
+
+    def close(self) -> None:
+        torch.cuda.current_stream(self.local[0].device).synchronize()
+        dist.barrier(group=self.group)  # no rank still reads a peer's buffer
+        self.records = None
+        torch.cuda.synchronize(self.local[0].device)
+        dist.barrier(group=self.group)
