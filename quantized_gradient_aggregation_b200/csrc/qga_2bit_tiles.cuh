@@ -225,21 +225,6 @@ __device__ __forceinline__ uint32_t quantize_word(float *__restrict__ residual,
     return word;
 }
 
-// Values of the 4 codes in a byte (first element in bits 7..6).
-__device__ __forceinline__ float4 tb_decode4(uint32_t byte, float neg, float pos)
-{
-    return make_float4(tb_value((byte >> 6) & 3u, neg, pos), tb_value((byte >> 4) & 3u, neg, pos),
-                       tb_value((byte >> 2) & 3u, neg, pos), tb_value(byte & 3u, neg, pos));
-}
-
-// The byte of group slot j of this lane, given the lane's own word of the
-// tile (word `lane` of the tile's 32 words).
-__device__ __forceinline__ uint32_t tb_group_byte(uint32_t my_word, int j, int lane)
-{
-    const uint32_t w = __shfl_sync(kFullMask, my_word, j * (kWarp / 4) + (lane >> 2));
-    return (w >> (24 - 8 * (lane & 3))) & 0xFFu;
-}
-
 // Store the 4 values of group gi of an fp32 output of n elements.
 template <bool kVec>
 __device__ __forceinline__ void store_group(float *__restrict__ out, int64_t n, int64_t gi, float4 v)
@@ -252,22 +237,6 @@ __device__ __forceinline__ void store_group(float *__restrict__ out, int64_t n, 
         for (int k = 0; k < 4; ++k)
             if (4 * gi + k < n)
                 st_stream_f1(out + 4 * gi + k, vv[k]);
-    }
-}
-
-// Dequantize tile `tile` of one record.
-template <bool kVec>
-__device__ __forceinline__ void dequantize_2bit_tile(const uint32_t *__restrict__ payload,
-                                                     float *__restrict__ out, int64_t n,
-                                                     int64_t tile, float neg, float pos, int lane)
-{
-    const int64_t nwords = (n + 15) >> 4;
-    const int64_t w = tile * kTileWords + lane;
-    const uint32_t my_word = w < nwords ? ld_stream_u32(payload + w) : 0u;
-#pragma unroll
-    for (int j = 0; j < kGroupsPerLane; ++j) {
-        const uint32_t byte = tb_group_byte(my_word, j, lane);
-        store_group<kVec>(out, n, tile * kTileGroups + j * kWarp + lane, tb_decode4(byte, neg, pos));
     }
 }
 
