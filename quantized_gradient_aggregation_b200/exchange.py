@@ -203,3 +203,46 @@ class PeerMergeExchange:
         self.records = None
         torch.cuda.synchronize(self.local[0].device)
         dist.barrier(group=self.group)
+
+
+class QsgdAllGather:
+    """One QSGD-MaxNorm exchange step across ranks, b bits per element.
+
+    ``step(grad, out)``: the local max |g| (``qga_qsgd_mn_max`` on this
+    rank's gradient), an all-reduce MAX of that one float, so that every rank
+    quantizes on the same global M; the quantize of this rank's gradient
+    with the seed ``seed_base + rank``; an all-gather of the W records; and
+    the integer-sum merge of the records in rank order into ``out``.  Every
+    rank ends with the same aggregate bit for bit.  QSGD-MaxNorm keeps no
+    residual.
+
+    ``ops`` replaces the library calls by ``(words(n, b), local_max(grad,
+    m_out), quantize(grad, compr, b, seed, m), merge(records, out, b))`` with
+    the same arguments, so that the step's ordering can be driven on a CPU
+    process group with stand-in arithmetic.
+    """
+
+    def __init__(self, n: int, bits: int, seed_base: int, group=None, *, device=None, ops=None):
+        from . import qga_qsgd_mn_dequant_accumulate, qga_qsgd_mn_max, qga_qsgd_mn_quantize, qga_qsgd_words
+        if ops is None:
+            ops = (qga_qsgd_words, lambda g, m: qga_qsgd_mn_max([g], m), qga_qsgd_mn_quantize,
+                   qga_qsgd_mn_dequant_accumulate)
+        words_fn, self._max, self._quantize, self._merge = ops
+        self.n = int(n)
+        self.bits = int(bits)
+        self.group = group
+        self.world = dist.get_world_size(group)
+        self.seed = int(seed_base) + dist.get_rank(group)
+        if device is None:
+            device = torch.device("cuda", torch.cuda.current_device())
+        self.words = int(words_fn(self.n, self.bits))
+        self.m = torch.zeros(1, dtype=torch.float32, device=device)
+        self.local = torch.empty(self.words, dtype=torch.int32, device=device)
+        self.gathered = torch.empty(self.world * self.words, dtype=torch.int32, device=device)
+
+    def step(self, grad: torch.Tensor, out: torch.Tensor) -> None:
+        self._max(grad, self.m)
+        dist.all_reduce(self.m, op=dist.ReduceOp.MAX, group=self.group)
+        self._quantize(grad, self.local, self.bits, self.seed, self.m)
+        records = gather_records(self.local, self.gathered, self.group)
+        self._merge(records, out, self.bits)

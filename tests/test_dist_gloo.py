@@ -230,3 +230,42 @@ def test_bucketed_exchange_distinct_ranks(world):
     """, world=world)
     sums = {o.strip().splitlines()[-1] for o in outs}
     assert len(sums) == 1 and next(iter(sums)).startswith("ok")
+
+
+@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("b", [2, 8])
+def test_qsgd_exchange_distinct_ranks(world, b):
+    """QSGD-MaxNorm across gloo ranks: every rank's local max, the all-reduce
+    MAX, each rank's own seed, the gather in rank order and the merge, with
+    the oracle's arithmetic injected (host tensors)."""
+    outs = _run_ranks(_EXCHANGE_PRELUDE + f"""
+    from quantized_gradient_aggregation_b200.exchange import QsgdAllGather
+    b, n, seed_base = {b}, 10_007, 1234
+
+    def local_max(g, m):
+        m.fill_(float(oracle.qsgd_mn_max([g.numpy()])))
+
+    def quantize(g, compr, bits, seed, m):
+        c = oracle.qsgd_mn_quantize(g.numpy(), bits, seed, np.float32(m.item()))
+        compr.copy_(torch.from_numpy(c.view(np.int32)))
+
+    def merge(records, out, bits):
+        out.copy_(torch.from_numpy(oracle.qsgd_mn_dequant_accumulate([as_u32(r) for r in records],
+                                                                   out.numel(), bits)))
+
+    ex = QsgdAllGather(n, b, seed_base, device="cpu", ops=(oracle.qsgd_words, local_max, quantize, merge))
+    out = torch.empty(n)
+    for step in range(2):
+        ex.step(torch.from_numpy(grad_of(rank, step, n)), out)
+        M = oracle.qsgd_mn_max([grad_of(k, step, n) for k in range(world)])
+        assert float(ex.m.item()) == float(M), step
+        recs = [oracle.qsgd_mn_quantize(grad_of(k, step, n), b, seed_base + k, M) for k in range(world)]
+        rows = as_u32(ex.gathered).reshape(world, -1)
+        for k in range(world):
+            assert np.array_equal(rows[k], recs[k]), (step, k)
+        want = oracle.qsgd_mn_dequant_accumulate(recs, n, b)
+        assert np.array_equal(out.numpy().view(np.uint32), want.view(np.uint32)), step
+    print("ok", float(out.abs().sum()))
+    """, world=world)
+    sums = {o.strip().splitlines()[-1] for o in outs}
+    assert len(sums) == 1 and next(iter(sums)).startswith("ok")

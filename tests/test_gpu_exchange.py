@@ -77,3 +77,25 @@ def test_bucketed_exchange_one_rank(nccl_group):
             assert same_bits_f32(f32(outs[b]), want), (it, b)
             for t in range(len(buckets[b])):
                 assert same_bits_f32(f32(res[b][t]), r_host[b][t]), (it, b, t)
+
+
+@pytest.mark.parametrize("b", [2, 4, 8])
+def test_qsgd_exchange_one_rank(nccl_group, b):
+    """QSGD-MaxNorm step on a one-rank NCCL group: the local max, its
+    all-reduce, the quantize with this rank's seed, the gather and the merge,
+    all on the device, against the oracle."""
+    from quantized_gradient_aggregation_b200.exchange import QsgdAllGather
+    n = 1_000_003
+    gen = torch.Generator(device=DEV)
+    gen.manual_seed(7 + b)
+    ex = QsgdAllGather(n, b, 1234)
+    out = torch.empty(n, device=DEV)
+    for it in range(2):
+        g = torch.randn(n, device=DEV, generator=gen) * 0.3
+        ex.step(g, out)
+        g_host = f32(g)
+        M = oracle.qsgd_mn_max([g_host])
+        assert ex.m.item() == M, it
+        rec = oracle.qsgd_mn_quantize(g_host, b, 1234, M)
+        assert np.array_equal(ex.gathered.cpu().numpy().view(np.uint32), rec), it
+        assert same_bits_f32(f32(out), oracle.qsgd_mn_dequant_accumulate([rec], n, b)), it

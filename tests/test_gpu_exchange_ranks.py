@@ -157,3 +157,30 @@ def test_bucketed_exchange_across_gpus(world):
     """, world)
     sums = {o.strip().splitlines()[-1] for o in outs}
     assert len(sums) == 1 and next(iter(sums)).startswith("ok")
+
+
+@pytest.mark.parametrize("world", _worlds())
+@pytest.mark.parametrize("b", [2, 8])
+def test_qsgd_exchange_across_gpus(world, b):
+    if torch.cuda.device_count() < world:
+        pytest.skip(f"needs {world} GPUs")
+    outs = _run_gpu_ranks(_PRELUDE + f"""
+    from quantized_gradient_aggregation_b200.exchange import QsgdAllGather
+    b, n, seed_base = {b}, 1_000_003, 1234
+    ex = QsgdAllGather(n, b, seed_base)
+    out = torch.empty(n, device=dev)
+    for step in range(2):
+        ex.step(torch.from_numpy(grad_of(rank, step, n)).to(dev), out)
+        torch.cuda.synchronize()
+        M = oracle.qsgd_mn_max([grad_of(k, step, n) for k in range(world)])
+        assert float(ex.m.item()) == float(M), step
+        recs = [oracle.qsgd_mn_quantize(grad_of(k, step, n), b, seed_base + k, M) for k in range(world)]
+        rows = u32(ex.gathered).reshape(world, -1)
+        for k in range(world):
+            assert np.array_equal(rows[k], recs[k]), (step, k)
+        want = oracle.qsgd_mn_dequant_accumulate(recs, n, b)
+        assert np.array_equal(u32(out), want.view(np.uint32)), step
+    print("ok", float(out.abs().sum()))
+    """, world)
+    sums = {o.strip().splitlines()[-1] for o in outs}
+    assert len(sums) == 1 and next(iter(sums)).startswith("ok")
