@@ -282,7 +282,7 @@ __device__ __forceinline__ void merge_store_word(LevelSum<B> &acc, int64_t kw, f
     }
 }
 
-// Any worker count (used for W > 8): batches of 8 workers, the payload
+// Any worker count (used for W > 16): batches of 8 workers, the payload
 // pointers read from the kernel's parameter space.  Measured at n = 2^27,
 // b = 4, W = 9 / 16 / 32: 212 / 279 / 467 us, against 230 / 312 / 533 us
 // with the pointers read back from shared memory in every iteration (b = 2
@@ -370,9 +370,14 @@ __global__ void __launch_bounds__(kThreads)
 #endif
 constexpr int kMergeWSlots = QGA_QSGD_MERGE_W_SLOTS;
 
-template <int B, bool kVec, int kW>
+// kPad: any W up to kW; the words of workers W .. kW - 1 are taken as 0, a
+// word of levels 0, which adds nothing to the sums (the bias it adds is the
+// one the offset removes for kW words).  Measured at n = 2^27, W = 16, b = 2
+// / 4 / 8: 180 / 262 / 423 us, against 222 / 277 / 470 us for the runtime-W
+// kernel.
+template <int B, bool kVec, int kW, bool kPad>
 __global__ void __launch_bounds__(kThreads, QGA_QSGD_MERGE_W_MIN_BLOCKS)
-    qsgd_merge_w_kernel(const __grid_constant__ RecordSet set, float *__restrict__ out, int64_t n)
+    qsgd_merge_w_kernel(const __grid_constant__ RecordSet set, int W, float *__restrict__ out, int64_t n)
 {
     constexpr int kSlots = kMergeWSlots;
     static_assert(kW >= 1 && kW <= LevelSum<B>::kBatchMax, "one batch fits the narrow lanes");
@@ -389,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, QGA_QSGD_MERGE_W_MIN_BLOCKS)
             const int64_t k = (sl * kSlots + s) * kWarp + lane;
 #pragma unroll
             for (int i = 0; i < kW; ++i)
-                wd[s][i] = k < nwords ? ld_stream_u32(set.rec[i] + 3 + k) : 0u;
+                wd[s][i] = ((!kPad || i < W) && k < nwords) ? ld_stream_u32(set.rec[i] + 3 + k) : 0u;
         }
 #pragma unroll
         for (int s = 0; s < kSlots; ++s) {
@@ -412,7 +417,7 @@ std::atomic<int> occ_qw[3][64];
 #define QGA_QSGD_LANE_WORDS 1
 #endif
 std::atomic<int> occ_m[3][2][64];
-std::atomic<int> occ_mw[3][2][9][64]; // [bits][vec][W][device]
+std::atomic<int> occ_mw[3][2][17][64]; // [bits][vec][W][device]
 
 int bits_slot(int bits) { return bits == 2 ? 0 : (bits == 4 ? 1 : (bits == 8 ? 2 : -1)); }
 
@@ -471,29 +476,30 @@ void launch_quantize(const float *grad, uint32_t *compr, int64_t n, uint64_t see
     }
 }
 
-template <int B, bool kVec, int kW>
-void launch_merge_w(const RecordSet &set, float *out, int64_t n, cudaStream_t stream)
+template <int B, bool kVec, int kW, bool kPad = false>
+void launch_merge_w(const RecordSet &set, int W, float *out, int64_t n, cudaStream_t stream)
 {
-    auto k = qsgd_merge_w_kernel<B, kVec, kW>;
+    auto k = qsgd_merge_w_kernel<B, kVec, kW, kPad>;
     const int64_t nwords = (n * B + 31) >> 5;
     const int64_t per_block = (int64_t)kThreads * kMergeWSlots;
     k<<<grid_for((nwords + per_block - 1) / per_block, resident_blocks(k, kThreads, occ_mw[bits_slot(B)][kVec][kW]),
                  kQsgdMergeWWaves),
-        kThreads, 0, stream>>>(set, out, n);
+        kThreads, 0, stream>>>(set, W, out, n);
 }
 
 template <int B, bool kVec>
 void launch_merge_w(const RecordSet &set, int W, float *out, int64_t n, cudaStream_t stream)
 {
     switch (W) {
-    case 1: launch_merge_w<B, kVec, 1>(set, out, n, stream); break;
-    case 2: launch_merge_w<B, kVec, 2>(set, out, n, stream); break;
-    case 3: launch_merge_w<B, kVec, 3>(set, out, n, stream); break;
-    case 4: launch_merge_w<B, kVec, 4>(set, out, n, stream); break;
-    case 5: launch_merge_w<B, kVec, 5>(set, out, n, stream); break;
-    case 6: launch_merge_w<B, kVec, 6>(set, out, n, stream); break;
-    case 7: launch_merge_w<B, kVec, 7>(set, out, n, stream); break;
-    default: launch_merge_w<B, kVec, 8>(set, out, n, stream); break;
+    case 1: launch_merge_w<B, kVec, 1>(set, W, out, n, stream); break;
+    case 2: launch_merge_w<B, kVec, 2>(set, W, out, n, stream); break;
+    case 3: launch_merge_w<B, kVec, 3>(set, W, out, n, stream); break;
+    case 4: launch_merge_w<B, kVec, 4>(set, W, out, n, stream); break;
+    case 5: launch_merge_w<B, kVec, 5>(set, W, out, n, stream); break;
+    case 6: launch_merge_w<B, kVec, 6>(set, W, out, n, stream); break;
+    case 7: launch_merge_w<B, kVec, 7>(set, W, out, n, stream); break;
+    case 8: launch_merge_w<B, kVec, 8>(set, W, out, n, stream); break;
+    default: launch_merge_w<B, kVec, 16, true>(set, W, out, n, stream); break; // 9 .. 16
     }
 }
 
@@ -501,7 +507,7 @@ template <int B>
 void launch_merge(const RecordSet &set, int W, float *out, int64_t n, cudaStream_t stream)
 {
     const int s = bits_slot(B);
-    if (W <= 8) {
+    if (W <= 16) {
         if (aligned(out, 32))
             launch_merge_w<B, true>(set, W, out, n, stream);
         else

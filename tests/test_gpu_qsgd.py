@@ -95,7 +95,7 @@ def test_quantize_misaligned_and_special(b):
 
 
 @pytest.mark.parametrize("b", BITS)
-@pytest.mark.parametrize("W", [1, 2, 3, 5, 7, 8, 9, 64])
+@pytest.mark.parametrize("W", [1, 2, 3, 5, 7, 8, 9, 12, 16, 17, 64])
 @pytest.mark.parametrize("n", [1, 17, 513, 65_537])
 def test_merge(b, W, n):
     q = qga()
@@ -121,7 +121,7 @@ def test_merge(b, W, n):
 
 
 @pytest.mark.parametrize("b", BITS)
-@pytest.mark.parametrize("W", [1, 2, 3, 4, 5, 6, 7, 8, 9, 17, 64])
+@pytest.mark.parametrize("W", [1, 2, 3, 4, 5, 6, 7, 8, 9, 11, 15, 16, 17, 64])
 def test_merge_random_records(b, W):
     """Arbitrary bit patterns as records (every b-bit field value, -2^(b-1)
     included, which no quantize writes) merge as the oracle merges them, for

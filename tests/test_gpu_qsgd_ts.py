@@ -92,7 +92,7 @@ def test_quantize_boundary_misaligned_and_special(b1, b2):
 
 
 @pytest.mark.parametrize("b1,b2", PAIRS)
-@pytest.mark.parametrize("W", [1, 2, 3, 5, 8, 9, 64])
+@pytest.mark.parametrize("W", [1, 2, 3, 5, 8, 9, 13, 16, 17, 64])
 @pytest.mark.parametrize("n", [1, 17, 513, 65_537])
 def test_merge(b1, b2, W, n):
     q = qga()
@@ -117,7 +117,7 @@ def test_merge(b1, b2, W, n):
 
 
 @pytest.mark.parametrize("b1,b2", [(2, 4), (4, 8), (8, 2)])
-@pytest.mark.parametrize("W", [1, 2, 3, 4, 5, 6, 7, 8, 9, 17])
+@pytest.mark.parametrize("W", [1, 2, 3, 4, 5, 6, 7, 8, 9, 12, 16, 17])
 def test_merge_random_records(b1, b2, W):
     """Arbitrary bit patterns in both sub-records (every level value, both
     signs, on both scales at once) merge as the oracle merges them, for every
