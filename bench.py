@@ -58,7 +58,7 @@ QUANT_SOURCES = ("qga_common.cuh", "qga_2bit_tiles.cuh", "qga_2bit.cu")
 QSGD_SOURCES = ("qga_common.cuh", "qga_qsgd_level.cuh", "qga_qsgd.cu")
 TS_SOURCES = ("qga_common.cuh", "qga_qsgd_level.cuh", "qga_qsgd_ts.cu")
 MEASURED_ALU = {
-    "f0cac2ee0dafa582": {"b2": 12.78, "b4": 12.88, "b8": 13.58},
+    "6043dbb4f8cc3ed9": {"b2": 12.78, "b4": 12.88, "b8": 13.58},
     "cec14726e428f3f1": {"b4_8": 23.03, "b2_4": 21.50},
 }
 ALU_CLOCK_MHZ = 1965.0   # clocks.max.sm of the B200
